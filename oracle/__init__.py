@@ -1,0 +1,229 @@
+"""fp64 CPU oracle for the RRAttention prefill operator.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code with
+the CUDA path (``dynamic_block_sparse_rr_b200``) and the CUDA path never calls it.
+
+It restates, plainly and slowly, what the method computes.  The source is the
+RRAttention abstract and TL;DR ("RRAttention: Dynamic Block Sparse Attention via
+Per-Head Round-Robin Shifts for Long-Context Inference", sciencestack.ai page:
+Abstract, TL;DR, Figure 2 and Figure 3 captions; the same abstract on the
+taxoreview, paperdot and fugumt pages).  The pages carry no equations and no
+algorithm box, so every definition below is the plainest reading of that text.
+The readings:
+
+R1  Sampling ("rotating query sampling positions across attention heads within
+    each stride"; title: "Per-Head Round-Robin Shifts").  Head h samples, in
+    stride i, the query at position p(h, i) = i*S + (h mod S).  The shift is
+    fixed per head; it does not rotate across strides.
+R2  Stride-level keys ("stride-level aggregation", cost O(L^2/S^2)).  The keys
+    of stride j are reduced to their mean, Kbar[j] = (1/S) sum_{t<S} K[j*S+t].
+    The O(L^2/S^2) cost needs the key side reduced by S as well; the mean keeps
+    every key's contribution while the queries stay real, unpooled rows
+    ("query independence").                                   [parity unpinned]
+R3  Scores.  s[h,i,j] = Qs[h,i] . Kbar[j, h/g] / sqrt(d) for stride-causal j <= i
+    (the diagonal stride is included, so a row is never empty).
+                                                              [parity unpinned]
+R4  Each sampled row is a softmax over its j <= i.
+R5  Block mass ("aggregates the scores to BxB blocks").  A query block I holds
+    the r = B/S sampled rows i with i*S in I, a key block J the r strides j
+    with j*S in J.  M[h,I,J] = sum_{i in I} sum_{j in J} P[h,i,j], normalised
+    per row: m[h,I,J] = M[h,I,J] / sum_{J' <= I} M[h,I,J'].
+R6  Adaptive Top-tau ("smallest set of key blocks whose normalised mass reaches
+    tau").  For each row I < Nb-1: order J in [0, I] by (m descending, J
+    ascending), keep the shortest prefix whose running sum is >= tau.  tau >= 1
+    keeps every J <= I.
+R7  Static protection of the last query block (TL;DR): the last row I = Nb-1
+    keeps every J <= Nb-1, for every tau.  No other block is forced.
+R8  Block-sparse causal attention ("computing only half of the attention
+    blocks").  Query q in block I attends, with softmax scale 1/sqrt(d), to
+    every key k <= q that lies in a selected block of row I.
+R9  Mask comparison band (tolerance of the operator's specification): a block
+    is near-threshold when the running sum just before or just after it, in
+    the R6 order, lies within `band` of tau; a near-tie is a pair of blocks at
+    the cut whose masses differ by less than `tie`.
+
+Pins (tests/test_oracle.py): R8 against torch's scaled_dot_product_attention in
+fp64 (tau = 1 and arbitrary block masks); R1-R5 at S = 1 against the exact
+full-attention block mass from the attention matrix that scaled_dot_product_
+attention returns; R3-R5 with all-zero keys against the closed form
+P[i,j] = 1/(i+1) (a hand-derived fixture in the Figure 2 configuration S=4,
+B=8); R6 against brute-force subset enumeration; R7 by inspection of every row.
+R2 and R3 for S > 1 have no pin beyond those reductions: "parity unpinned".
+
+All arithmetic is float64.  Inputs are the bf16 values both paths receive,
+widened exactly.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+# ---------------------------------------------------------------- R1 sampling
+def sampled_positions(L: int, H: int, S: int) -> np.ndarray:
+    """p[h, i] = i*S + (h mod S), shape [H, L/S] (R1)."""
+    Ns = L // S
+    i = np.arange(Ns, dtype=np.int64)
+    return np.stack([i * S + (h % S) for h in range(H)])
+
+
+# ------------------------------------------------------------ R2 stride keys
+def pool_keys(K: np.ndarray, S: int) -> np.ndarray:
+    """Kbar[j, kv, :] = mean over the S keys of stride j (R2).  K: [L, Hkv, d]."""
+    L, Hkv, d = K.shape
+    return K.reshape(L // S, S, Hkv, d).mean(axis=1)
+
+
+# ------------------------------------------------------- R3-R5 block masses
+def block_mass(Q: np.ndarray, K: np.ndarray, B: int, S: int, row_chunk: int = 2048) -> np.ndarray:
+    """Unnormalised block mass M[h, I, J] (R3-R5), zero above the diagonal.
+
+    Q: [L, H, d], K: [L, Hkv, d] (float64).  Returns [H, Nb, Nb] float64.
+    """
+    L, H, d = Q.shape
+    Hkv = K.shape[1]
+    g = H // Hkv
+    Ns, Nb, r = L // S, L // B, B // S
+    Kbar = pool_keys(K, S)
+    pos = sampled_positions(L, H, S)
+    scale = 1.0 / math.sqrt(d)
+    M = np.zeros((H, Nb, Nb), dtype=np.float64)
+    step = max(r, (row_chunk // r) * r)
+    for h in range(H):
+        Qs = Q[pos[h], h, :]                     # [Ns, d] real sampled queries
+        Kb = Kbar[:, h // g, :]                  # [Ns, d]
+        for a in range(0, Ns, step):
+            b = min(Ns, a + step)
+            s = (Qs[a:b] @ Kb[:b].T) * scale     # rows i in [a,b), strides j < b
+            i_idx = np.arange(a, b)[:, None]
+            j_idx = np.arange(b)[None, :]
+            s = np.where(j_idx <= i_idx, s, -np.inf)
+            s = s - s.max(axis=1, keepdims=True)
+            P = np.exp(s)
+            P = P / P.sum(axis=1, keepdims=True)   # R4
+            nI, nJ = (b - a) // r, b // r
+            M[h, a // r:a // r + nI, :nJ] += P.reshape(nI, r, nJ, r).sum(axis=(1, 3))
+    return M
+
+
+def normalise_mass(M: np.ndarray) -> np.ndarray:
+    """m[h, I, J] = M[h, I, J] / sum_{J' <= I} M[h, I, J'] (R5); zero above the diagonal."""
+    H, Nb, _ = M.shape
+    tri = np.tril(np.ones((Nb, Nb), dtype=bool))
+    Mt = np.where(tri[None], M, 0.0)
+    return Mt / Mt.sum(axis=2, keepdims=True)
+
+
+# ---------------------------------------------------------- R6/R7 selection
+def sorted_order(m_row: np.ndarray) -> np.ndarray:
+    """J order by mass descending, then J ascending (R6)."""
+    n = m_row.shape[0]
+    return np.lexsort((np.arange(n), -m_row))
+
+
+def top_tau_row(m_row: np.ndarray, I: int, Nb: int, tau: float) -> np.ndarray:
+    """Selected key blocks of row I, ascending (R6, R7).  m_row: masses of J = 0..I."""
+    n = I + 1
+    if tau >= 1.0 or I == Nb - 1:
+        return np.arange(n, dtype=np.int32)
+    order = sorted_order(m_row[:n])
+    run = np.cumsum(m_row[:n][order])
+    hit = np.nonzero(run >= tau)[0]
+    k = int(hit[0]) + 1 if hit.size else n
+    return np.sort(order[:k]).astype(np.int32)
+
+
+def select(m: np.ndarray, tau: float):
+    """count [H, Nb] int32 and idx [H, Nb, Nb] int32 (ascending, -1 past count)."""
+    H, Nb, _ = m.shape
+    count = np.zeros((H, Nb), dtype=np.int32)
+    idx = np.full((H, Nb, Nb), -1, dtype=np.int32)
+    for h in range(H):
+        for I in range(Nb):
+            sel = top_tau_row(m[h, I], I, Nb, tau)
+            count[h, I] = sel.size
+            idx[h, I, :sel.size] = sel
+    return count, idx
+
+
+def rr_search(Q: np.ndarray, K: np.ndarray, B: int, S: int, tau: float):
+    """The pattern search: returns (count, idx, m) with m the normalised block mass."""
+    m = normalise_mass(block_mass(Q, K, B, S))
+    count, idx = select(m, tau)
+    return count, idx, m
+
+
+def full_causal_mask(H: int, Nb: int):
+    """Every causal block selected (the tau >= 1 mask)."""
+    count = np.tile(np.arange(1, Nb + 1, dtype=np.int32), (H, 1))
+    idx = np.tile(np.where(np.tri(Nb, dtype=bool), np.arange(Nb)[None, :], -1).astype(np.int32),
+                  (H, 1, 1))
+    return count, idx
+
+
+# ------------------------------------------------------ R8 sparse attention
+def sparse_attention_block(Q, K, V, h: int, I: int, blocks, B: int) -> np.ndarray:
+    """Output rows of query block I, head h, over the listed key blocks (R8).
+
+    Returns [B, d] float64.
+    """
+    L, H, d = Q.shape
+    g = H // K.shape[1]
+    kv = h // g
+    blocks = np.asarray(blocks, dtype=np.int64)
+    keys = (blocks[:, None] * B + np.arange(B)[None, :]).reshape(-1)
+    q_pos = I * B + np.arange(B)
+    s = (Q[q_pos, h, :] @ K[keys, kv, :].T) / math.sqrt(d)
+    s = np.where(keys[None, :] <= q_pos[:, None], s, -np.inf)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=1, keepdims=True)
+    return p @ V[keys, kv, :]
+
+
+def sparse_attention(Q, K, V, count, idx, B: int, rows=None) -> np.ndarray:
+    """Block-sparse causal attention (R8).
+
+    rows: None for every (h, I), else an iterable of (h, I); rows not computed
+    stay NaN.  Returns [L, H, d] float64.
+    """
+    L, H, d = Q.shape
+    Nb = L // B
+    O = np.full((L, H, d), np.nan, dtype=np.float64)
+    if rows is None:
+        rows = [(h, I) for h in range(H) for I in range(Nb)]
+    for h, I in rows:
+        c = int(count[h, I])
+        O[I * B:(I + 1) * B, h, :] = sparse_attention_block(Q, K, V, h, I, idx[h, I, :c], B)
+    return O
+
+
+# -------------------------------------------------------- R9 comparison band
+def band_blocks(m_row: np.ndarray, I: int, tau: float, band: float = 1e-4, tie: float = 1e-6):
+    """Blocks of row I whose selection may legitimately differ (R9).
+
+    Returns (near_threshold, near_tie): two sets of J.  near_threshold: the
+    running sum (R6 order) just before or just after the block lies within
+    `band` of tau.  near_tie: blocks at the cut whose mass is within `tie` of
+    the mass of the block on the other side of the cut.
+    """
+    n = I + 1
+    order = sorted_order(m_row[:n])
+    vals = m_row[:n][order]
+    run = np.cumsum(vals)
+    before = np.concatenate([[0.0], run[:-1]])
+    near = set(int(order[t]) for t in range(n)
+               if abs(before[t] - tau) <= band or abs(run[t] - tau) <= band)
+    hit = np.nonzero(run >= tau)[0]
+    k = int(hit[0]) + 1 if hit.size else n
+    ties = set()
+    if 0 < k < n:
+        cut_in, cut_out = vals[k - 1], vals[k]
+        for t in range(n):
+            if t < k and abs(vals[t] - cut_out) < tie:
+                ties.add(int(order[t]))
+            if t >= k and abs(vals[t] - cut_in) < tie:
+                ties.add(int(order[t]))
+    return near, ties
