@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Benchmark of the RRAttention prefill operator (search + block-sparse attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one attention layer's synthetic
+inputs: key pooling, the round-robin sampled-score search, Top-tau selection and
+the block-sparse attention, through the C ABI.  Default workload: the 128K
+LLaMA-3.1-8B-shaped GQA layer (H=32, Hkv=8, d=128, L=131072, B=128, S=16,
+tau=0.95, planted sinks + local band).
+
+One JSON line (rank 0).  `value` is TFLOP/s over the visited blocks
+(4*B*B*d flops per visited block, diagonal blocks counted in full), summed over
+ranks and divided by the slowest rank's device time.  Under torchrun every rank
+runs its own independent layer (weak scaling, no collective on the data path).
+
+`--impl reference` times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only) and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gen  # noqa: E402
+
+METRIC = "sparse prefill attn ms & TFLOP/s at 128K (search+attn); speedup vs dense"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "bsfa_llama128k_traffic.txt")
+
+
+def workload_config(cfg: gen.Config, tau: float) -> dict:
+    return {"workload": f"{cfg.name}: GQA attention layer H={cfg.H}/Hkv={cfg.Hkv}, d={cfg.d}, L={cfg.L}, "
+                        f"B={cfg.B}, S={cfg.S}, tau={tau}, batch 1",
+            "structure": {0: "iid", 1: "planted sinks", 2: "planted sinks + local band", 3: "video frames"}[
+                cfg.structure],
+            "L": cfg.L, "H": cfg.H, "Hkv": cfg.Hkv, "d": cfg.d, "B": cfg.B, "S": cfg.S, "tau": tau,
+            "l2": "inputs exceed L2 (q alone is %.2f GB > 126 MB)" % (cfg.L * cfg.H * cfg.d * 2 / 1e9),
+            "seed": cfg.seed}
+
+
+def block_flops(cfg: gen.Config, visited_blocks: int) -> float:
+    return 4.0 * cfg.B * cfg.B * cfg.d * visited_blocks
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"bf16_tflops": d["bf16_tflops"], "bf16_tflops_sustained": d.get("bf16_tflops_sustained"),
+                "hbm_gbs": d["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_traffic_bytes():
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    src = os.path.join(ROOT, "dynamic_block_sparse_rr_b200", "csrc", "bsfa.cu")
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(PROFILE_TRAFFIC):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("bsfa_cu_sha256_16") != digest:
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch_full"])
+    except (KeyError, ValueError):
+        return None
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(cfg: gen.Config, tau: float, q, k, v, heads=1, rows_per_head=12, seed=0):
+    """Time the oracle on a bounded sample and extrapolate to one full step.
+
+    Sample: the full search for `heads` heads (every sampled row of the head) and
+    the sparse attention of `rows_per_head` query-block rows of each of those
+    heads, over the oracle's own mask.  Full-step time = search time x H/heads +
+    attention time / (visited blocks of the sampled rows) x (visited blocks of
+    the whole layer, estimated from the sampled heads' masks x H/heads).
+    """
+    import oracle
+    Nb = cfg.L // cfg.B
+    g = cfg.H // cfg.Hkv
+    rng = np.random.default_rng(seed)
+    t_search = t_attn = 0.0
+    blocks_sampled = blocks_head_total = 0
+    for hs in range(heads):
+        h = (hs * 7) % cfg.H
+        kv = h // g
+        Qh = gen.bf16_bits_to_f32(q[:, h:h + 1, :])
+        Kh = gen.bf16_bits_to_f32(k[:, kv:kv + 1, :])
+        Vh = gen.bf16_bits_to_f32(v[:, kv:kv + 1, :])
+        t0 = time.perf_counter()
+        count, idx, _ = oracle.rr_search(Qh, Kh, cfg.B, cfg.S, tau)
+        t_search += time.perf_counter() - t0
+        blocks_head_total += int(count.sum())
+        rows = sorted(set([Nb - 1] + [int(x) for x in rng.integers(0, Nb, rows_per_head - 1)]))
+        t0 = time.perf_counter()
+        for I in rows:
+            oracle.sparse_attention_block(Qh, Kh, Vh, 0, I, idx[0, I, :count[0, I]], cfg.B)
+        t_attn += time.perf_counter() - t0
+        blocks_sampled += int(sum(count[0, I] for I in rows))
+    scale_heads = cfg.H / heads
+    total_blocks = blocks_head_total * scale_heads
+    step_s = t_search * scale_heads + t_attn / max(blocks_sampled, 1) * total_blocks
+    flops = block_flops(cfg, total_blocks)
+    return {
+        "value": flops / step_s / 1e12,
+        "unit": "TFLOP/s",
+        "cores": blas_threads(),
+        "kind": "oracle",
+        "sample": (f"fp64 numpy oracle: full search of {heads} head(s) + attention of "
+                   f"{rows_per_head} query-block rows per sampled head ({blocks_sampled} visited blocks), "
+                   f"extrapolated to all {cfg.H} heads / {int(total_blocks)} visited blocks; "
+                   f"measured {t_search + t_attn:.1f} s, extrapolated step {step_s:.1f} s"),
+        "step_s": step_s,
+        "measured_s": t_search + t_attn,
+    }
+
+
+def run_reference(args, cfg, tau, world):
+    q, k, v = gen.make_config(cfg)
+    times = []
+    res = None
+    for it in range(args.warmup + args.steps):
+        res = oracle_sample(cfg, tau, q, k, v, heads=1, rows_per_head=args.ref_rows, seed=it)
+        if it >= args.warmup:
+            times.append(res["step_s"])
+    step_s = statistics.mean(times)
+    flops_per_step = res["value"] * 1e12 * res["step_s"]   # extrapolated work of one full step
+    value = flops_per_step / step_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg, tau),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"], "kind": "oracle",
+                         "sample": res["sample"] + "; each step is one such sample"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"rr_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args, cfg, tau, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import dynamic_block_sparse_rr_b200 as rr
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    q, k, v = gen.make_config(cfg, seed=cfg.seed + rank)
+    to_pinned = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    qh, kh, vh = to_pinned(q), to_pinned(k), to_pinned(v)
+    qd, kd, vd = qh.to(dev), kh.to(dev), vh.to(dev)
+    L, H, Hkv, d, B, S = cfg.L, cfg.H, cfg.Hkv, cfg.d, cfg.B, cfg.S
+    Nb = L // B
+    ws = rr.workspace(L, H, Hkv, d, B, S, dev)
+    count, idx = rr.empty_mask(H, Nb, dev)
+    o = torch.empty_like(qd)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        rr.search(qd, kd, B, S, tau, count=count, idx=idx, ws=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        rr.sparse_attn(qd, kd, vd, count, idx, B, out=o, ws=ws)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if rr.check_status(ws) != rr.RR_OK:
+        raise RuntimeError("device-side status after warm-up: %d" % rr.check_status(ws))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    status = rr.check_status(ws)
+    if status != rr.RR_OK:
+        raise RuntimeError("device-side status %d" % status)
+    total_ms = t_start.elapsed_time(t_end)
+    search_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    visited = int(count.sum().item())
+    flops = block_flops(cfg, visited)
+    gpu_launches = 4 * args.steps   # pool, search, top-tau, attention per step
+
+    # max over ranks of the timed region; sum of the work
+    tot = torch.tensor([total_ms, flops], dtype=torch.float64, device=dev)
+    if world > 1:
+        mx = tot.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = tot.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        total_ms_max, flops_all = float(mx[0]), float(sm[1])
+    else:
+        total_ms_max, flops_all = total_ms, flops
+    ms_per_step = total_ms_max / args.steps
+    value = flops_all / (ms_per_step / 1e3) / 1e12
+
+    # dense baseline: the same attention kernel with every causal block on
+    dense_ms = None
+    if not args.no_dense:
+        cd, idd = rr.empty_mask(H, Nb, dev)
+        rr.search(qd, kd, B, S, 1.0, count=cd, idx=idd, ws=ws)
+        rr.sparse_attn(qd, kd, vd, cd, idd, B, out=o, ws=ws)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 2
+        e0.record(stream)
+        for _ in range(reps):
+            rr.sparse_attn(qd, kd, vd, cd, idd, B, out=o, ws=ws)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        dense_ms = e0.elapsed_time(e1) / reps
+        dense_blocks = H * Nb * (Nb + 1) // 2
+        dense_tflops = block_flops(cfg, dense_blocks) / (dense_ms / 1e3) / 1e12
+        del cd, idd
+
+    # end to end through the public API with host buffers
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, min(args.steps, 2))
+    qd2, kd2, vd2 = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        qd2.copy_(qh, non_blocking=True)
+        kd2.copy_(kh, non_blocking=True)
+        vd2.copy_(vh, non_blocking=True)
+        rr.attention(qd2, kd2, vd2, B, S, tau, out=o, count=count, idx=idx, ws=ws)
+        oh.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = flops_all / (float(e2e_t[0]) / 1e3) / 1e12
+    h2d = (qh.numel() + kh.numel() + vh.numel()) * 2
+    d2h = oh.numel() * 2
+    del qd2, kd2, vd2
+
+    peaks = measured_peaks()
+    peak = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
+    achieved = flops / (attn_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": kernel_traffic_bytes(), "kernel": "bsfa_kernel<128,128>",
+                "peak_kind": f"bf16 dense, sustained ({peaks['source']})"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res = oracle_sample(cfg, tau, q, k, v, heads=1, rows_per_head=args.ref_rows)
+        cpu = {k2: res[k2] for k2 in ("value", "unit", "cores", "kind", "sample")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator, planted structure)",
+            "config": workload_config(cfg, tau),
+            "search_ms": search_ms, "attn_ms": attn_ms, "search_share": search_ms / (search_ms + attn_ms),
+            "dense_attn_ms": dense_ms, "dense_attn_tflops": dense_tflops if dense_ms else None,
+            "speedup_vs_dense": (dense_ms / ms_per_step) if dense_ms else None,
+            "visited_blocks": visited, "visited_fraction": visited / (H * Nb * (Nb + 1) / 2),
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": float(e2e_t[0]),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": gpu_launches, "clocks": clk, "roofline": roofline, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="llama128k", choices=sorted(gen.CONFIGS))
+    ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--ref-rows", type=int, default=12)
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("note: fewer than 3 warm-up steps requested", file=sys.stderr)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = gen.CONFIGS[args.config]
+    tau = args.tau if args.tau is not None else cfg.tau
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, cfg, tau, world)
+        return
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, cfg, tau, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

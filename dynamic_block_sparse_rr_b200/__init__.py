@@ -1,0 +1,158 @@
+"""Python binding of the B200 RRAttention prefill operator (``librr.so``).
+
+Argument marshalling only: every step of the operator runs in the CUDA kernels
+behind the C ABI of ``include/rr.h``.  PyTorch supplies device memory and the
+current stream.  There is no fallback: if ``librr.so`` is missing or cannot be
+loaded, importing the operator functions raises.
+
+Tensors: q ``[L, H, d]``, k and v ``[L, Hkv, d]``, bf16, contiguous, on one CUDA
+device.  Masks: ``count [H, Nb]`` and ``idx [H, Nb, Nb]`` int32 (see rr.h).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librr.so")
+
+RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT = range(6)
+
+# every symbol that include/rr.h declares
+EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status",
+           "rr_set_wait_limit_ns", "rr_status_string")
+
+
+class RRError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"librr.so not built at {LIB_PATH}; run python -m dynamic_block_sparse_rr_b200._build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.rr_workspace_size.argtypes = [i, i, i, i, i, i, ctypes.POINTER(sz)]
+        L.rr_search.argtypes = [vp, vp, i, i, i, i, i, i, f, vp, vp, vp, vp, sz, vp]
+        L.rr_sparse_attn.argtypes = [vp, vp, vp, i, i, i, i, i, vp, vp, vp, vp, sz, vp]
+        L.rr_attention.argtypes = [vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp, vp, sz, vp]
+        L.rr_check_status.argtypes = [vp, vp]
+        L.rr_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.rr_set_wait_limit_ns.restype = ctypes.c_uint64
+        L.rr_status_string.argtypes = [i]
+        L.rr_status_string.restype = ctypes.c_char_p
+        for name in ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().rr_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != RR_OK:
+        raise RRError(code, where)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _shape(q, k):
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("q must be [L, H, d] and k [L, Hkv, d]")
+    L, H, d = q.shape
+    if k.shape[0] != L or k.shape[2] != d:
+        raise ValueError("q and k disagree on L or d")
+    for t in (q, k):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    return L, H, k.shape[1], d
+
+
+def workspace_size(L: int, H: int, Hkv: int, d: int, B: int, S: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().rr_workspace_size(L, H, Hkv, d, B, S, ctypes.byref(n)), "rr_workspace_size")
+    return n.value
+
+
+def workspace(L: int, H: int, Hkv: int, d: int, B: int, S: int, device=None) -> torch.Tensor:
+    """A device workspace (uint8) of the size the operator needs."""
+    return torch.empty(workspace_size(L, H, Hkv, d, B, S), dtype=torch.uint8, device=device or "cuda")
+
+
+def empty_mask(H: int, Nb: int, device=None):
+    dev = device or "cuda"
+    return (torch.empty((H, Nb), dtype=torch.int32, device=dev),
+            torch.empty((H, Nb, Nb), dtype=torch.int32, device=dev))
+
+
+def search(q, k, B: int, S: int, tau: float, count=None, idx=None, mass=None, ws=None, stream=None):
+    """Pattern search -> (count [H, Nb], idx [H, Nb, Nb]).  ``mass`` (optional, fp32
+    [H, Nb, Nb]) receives the unnormalised block masses."""
+    L, H, Hkv, d = _shape(q, k)
+    Nb = L // B
+    if count is None or idx is None:
+        count, idx = empty_mask(H, Nb, q.device)
+    if ws is None:
+        ws = workspace(L, H, Hkv, d, B, S, q.device)
+    _check(lib().rr_search(q.data_ptr(), k.data_ptr(), L, H, Hkv, d, B, S, float(tau), count.data_ptr(),
+                           idx.data_ptr(), _ptr(mass), ws.data_ptr(), ws.numel(), _stream(stream)), "rr_search")
+    return count, idx
+
+
+def sparse_attn(q, k, v, count, idx, B: int, out=None, ws=None, stream=None):
+    """Causal block-sparse attention over (count, idx) -> o [L, H, d] bf16."""
+    L, H, Hkv, d = _shape(q, k)
+    _shape(v, k)
+    if out is None:
+        out = torch.empty_like(q)
+    if ws is None:
+        ws = torch.empty(256, dtype=torch.uint8, device=q.device)
+    _check(lib().rr_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), L, H, Hkv, d, B, count.data_ptr(),
+                                idx.data_ptr(), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "rr_sparse_attn")
+    return out
+
+
+def attention(q, k, v, B: int, S: int, tau: float, out=None, count=None, idx=None, ws=None, stream=None):
+    """Search then sparse attention on one stream -> (o, count, idx)."""
+    L, H, Hkv, d = _shape(q, k)
+    _shape(v, k)
+    Nb = L // B
+    if out is None:
+        out = torch.empty_like(q)
+    if count is None or idx is None:
+        count, idx = empty_mask(H, Nb, q.device)
+    if ws is None:
+        ws = workspace(L, H, Hkv, d, B, S, q.device)
+    _check(lib().rr_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), L, H, Hkv, d, B, S, float(tau),
+                              count.data_ptr(), idx.data_ptr(), out.data_ptr(), ws.data_ptr(), ws.numel(),
+                              _stream(stream)), "rr_attention")
+    return out, count, idx
+
+
+def check_status(ws, stream=None) -> int:
+    """Synchronise and return the device-side status of the last call on ``ws``."""
+    return lib().rr_check_status(ws.data_ptr(), _stream(stream))
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    return lib().rr_set_wait_limit_ns(int(ns))

@@ -1,0 +1,374 @@
+// bsfa.cu — causal block-sparse FlashAttention forward over the selected
+// blocks (RRAttention abstract: "computing only half of the attention
+// blocks", "2.4x speedup at 128K"; Figure 2 stage 3; Figure 3a).
+//
+// One CTA per (head h, query block I): a 128-row query tile (the B = 64 case
+// uses the first 64 rows), the key blocks J listed for (h, I) visited in
+// ascending order.  Both contractions per block run on tcgen05 with fp32
+// accumulators in TMEM:
+//     S = Q K_J^T           (A = Q, B = K_J from shared memory, K-major)
+//     O += P V_J            (A = P from TMEM as bf16, B = V_J, MN-major)
+// The block list is split between two softmax warpgroups (even / odd list
+// positions), each with its own S buffer and O accumulator, so the tensor core
+// works on one group's blocks while the other group runs its softmax.  Each
+// group keeps its own running max / sum; the two partial results are merged
+// exactly in the epilogue:  O = (O_a 2^(m_a-m) + O_b 2^(m_b-m)) / (l_a 2^(m_a-m)
+// + l_b 2^(m_b-m)).
+//
+// Online softmax in the exp2 domain with a lazy rescale: the running max is
+// only moved (and O rescaled in TMEM) when a row's new max exceeds it by more
+// than 8 (a factor 256), which keeps P <= 256 and is exact after the final
+// division because P and l always use the same max.
+//
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer (one
+// thread; owns the 512-column TMEM allocation), warps 2-5 softmax group 0,
+// warps 6-9 softmax group 1.  TMEM columns: S_0 [0,128), S_1 [128,256),
+// O_0 [256,384), O_1 [384,512); P_x overwrites the first B/2 columns of S_x.
+// K/V tiles stream through a 4-stage shared-memory ring in the order the MMA
+// consumes them: K0, K1, V0, K2, V1, K3, ...
+#include <cuda_bf16.h>
+
+#include "rr_internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace rr {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kStages = 4;
+
+template <int BN, int D>
+struct FaCfg {
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kTileBytes = BN * D * 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kStageOff = kQBytes;
+  static constexpr int kListOff = kStageOff + kStages * kTileBytes;
+  static constexpr int kCtrlOff = kListOff + kMaxBlocks * 4;
+  static constexpr int kUsed = kCtrlOff + 2048 + 1024;
+  // At least ~120 KB so that one CTA holds an SM (it allocates all 512 TMEM columns).
+  static constexpr int kSmem = kUsed > 122880 ? kUsed : 122880;
+};
+
+struct FaCtrl {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t merge;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  float2 ml[2][128];
+};
+
+template <int BN, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bsfa_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                const __grid_constant__ CUtensorMap mv, const int32_t* __restrict__ count,
+                const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int H, int Hkv, int Nb,
+                float sl2, unsigned int* status, uint64_t limit_ns) {
+  using C = FaCfg<BN, D>;
+  constexpr uint32_t kIdS = idesc_bf16_f32(128, BN, false, false);
+  constexpr uint32_t kIdO = idesc_bf16_f32(128, D, false, true);
+  constexpr float kRescale = 8.0f;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::kQOff;
+  uint8_t* sStage = smem + C::kStageOff;
+  int32_t* sList = reinterpret_cast<int32_t*>(smem + C::kListOff);
+  FaCtrl* ctl = reinterpret_cast<FaCtrl*>(smem + C::kCtrlOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int I = Nb - 1 - static_cast<int>(blockIdx.x / H);   // longer rows first
+  const int h = static_cast<int>(blockIdx.x % H);
+  const int kvh = h / (H / Hkv);
+  const long long row_id = static_cast<long long>(h) * Nb + I;
+  int cnt = count[row_id];
+  cnt = cnt < 0 ? 0 : (cnt > Nb ? Nb : cnt);
+  const int32_t* list = idx + row_id * Nb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 1);
+    }
+    mbar_init(smem_u32(&ctl->q_full), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(smem_u32(&ctl->s_full[x]), 1);
+      mbar_init(smem_u32(&ctl->p_full[x]), 128);
+    }
+    mbar_init(smem_u32(&ctl->merge), 256);
+    mbar_init(smem_u32(&ctl->drain), 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = ctl->tmem_base;
+  const Guard guard{&ctl->abort, status, limit_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && cnt > 0) {
+      tma_prefetch_desc(&mq);
+      tma_prefetch_desc(&mk);
+      tma_prefetch_desc(&mv);
+      const uint32_t qb = smem_u32(&ctl->q_full);
+      mbar_expect_tx(qb, C::kQBytes);
+      for (int a = 0; a < D / 64; ++a) tma_load_3d(smem_u32(sQ + a * 128 * 128), &mq, qb, a * 64, h, I * BN);
+    }
+    // the block list, read coalesced into shared memory
+    for (int t = lane; t < cnt; t += 32) sList[t] = __ldg(list + t);
+    __syncwarp();
+    if (lane == 0 && cnt > 0) {
+      int k = 0;
+      bool ok = true;
+      auto load = [&](const CUtensorMap* m, int J) {
+        const int st = k % kStages;
+        if (!wait_bar(smem_u32(&ctl->empty[st]), ((k / kStages) & 1) ^ 1, guard, 1)) return false;
+        const uint32_t fb = smem_u32(&ctl->full[st]);
+        mbar_expect_tx(fb, C::kTileBytes);
+        uint8_t* dst = sStage + st * C::kTileBytes;
+        for (int a = 0; a < D / 64; ++a) tma_load_3d(smem_u32(dst + a * BN * 128), m, fb, a * 64, kvh, J * BN);
+        ++k;
+        return true;
+      };
+      ok = load(&mk, sList[0]);
+      if (ok && cnt > 1) ok = load(&mk, sList[1]);
+      for (int t = 0; t < cnt && ok; ++t) {
+        ok = load(&mv, sList[t]);
+        if (ok && t + 2 < cnt) ok = load(&mk, sList[t + 2]);
+      }
+      drain_bar(smem_u32(&ctl->q_full), 0, kDrainLimitNs);
+      for (int kk = (k > kStages ? k - kStages : 0); kk < k; ++kk)
+        drain_bar(smem_u32(&ctl->full[kk % kStages]), (kk / kStages) & 1, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && cnt > 0) {
+      int k = 0;
+      bool ok = wait_bar(smem_u32(&ctl->q_full), 0, guard, 2);
+      tc_fence_after();
+      auto issue_s = [&](int x) {
+        const int st = k % kStages;
+        if (!wait_bar(smem_u32(&ctl->full[st]), (k / kStages) & 1, guard, 3)) return false;
+        tc_fence_after();
+        const uint8_t* kt = sStage + st * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(smem_u32(sQ + (kk >> 2) * 128 * 128 + 32 * (kk & 3)), 16, 1024);
+          const uint64_t bd = sdesc_sw128(smem_u32(kt + (kk >> 2) * BN * 128 + 32 * (kk & 3)), 16, 1024);
+          umma_ss(tm + x * 128, ad, bd, kIdS, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(smem_u32(&ctl->empty[st]));
+        ++k;
+        return true;
+      };
+      auto issue_pv = [&](int x, bool acc) {
+        const int st = k % kStages;
+        if (!wait_bar(smem_u32(&ctl->full[st]), (k / kStages) & 1, guard, 4)) return false;
+        tc_fence_after();
+        const uint8_t* vt = sStage + st * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(smem_u32(vt + kk * 16 * 128), BN * 128, 1024);
+          umma_ts(tm + 256 + x * 128, tm + x * 128 + kk * 8, bd, kIdO, (acc || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(smem_u32(&ctl->empty[st]));
+        ++k;
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok) umma_commit(smem_u32(&ctl->s_full[0]));
+      if (ok && cnt > 1) {
+        ok = issue_s(1);
+        if (ok) umma_commit(smem_u32(&ctl->s_full[1]));
+      }
+      for (int t = 0; t < cnt && ok; ++t) {
+        const int x = t & 1, u = t >> 1;
+        if (!wait_bar(smem_u32(&ctl->p_full[x]), u & 1, guard, 5)) { ok = false; break; }
+        tc_fence_after();
+        ok = issue_pv(x, u > 0);
+        if (ok && t + 2 < cnt) ok = issue_s(x);
+        if (ok) umma_commit(smem_u32(&ctl->s_full[x]));
+      }
+      umma_commit(smem_u32(&ctl->drain));
+      drain_bar(smem_u32(&ctl->drain), 0, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax groups
+    const int x = (warp - 2) >> 2;              // group 0: warps 2-5, group 1: warps 6-9
+    const int wq = warp & 3;                    // TMEM lane quarter
+    const int row = wq * 32 + lane;             // row of the query tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_col = tm + lane_off + x * 128;
+    const uint32_t o_col = tm + lane_off + 256 + x * 128;
+    const int n_a = (cnt + 1) >> 1, n_b = cnt >> 1;
+    const int n_x = x == 0 ? n_a : n_b;
+    const bool diag_last = cnt > 0 && __ldg(list + cnt - 1) == I;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int u = 0; u < n_x; ++u) {
+      const int t = 2 * u + x;
+      if (!wait_bar_warp(smem_u32(&ctl->s_full[x]), u & 1, guard, 6)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t raw[BN];
+      if constexpr (BN == 128) {
+        tmem_ld128(s_col, raw);
+      } else {
+        tmem_ld32x2(s_col, s_col + 32, raw);
+      }
+      float s[BN];
+      const bool diag = diag_last && t == cnt - 1;
+#pragma unroll
+      for (int j = 0; j < BN; ++j) s[j] = (diag && j > row) ? -INFINITY : __uint_as_float(raw[j]);
+      float mx = s[0];
+#pragma unroll
+      for (int j = 1; j < BN; ++j) mx = fmaxf(mx, s[j]);
+      const float m_blk = mx * sl2;
+      // lazy rescale: move the running max only when it grows by more than 2^8
+      bool rescale = false;
+      float alpha = 1.0f;
+      if (u == 0) {
+        m_run = m_blk;
+      } else {
+        const bool need = m_blk > m_run + kRescale;
+        rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+          alpha = ex2(m_run - m_blk);
+          l_run *= alpha;
+          m_run = m_blk;
+        }
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = ex2(fmaf(s[c * 32 + 2 * j], sl2, -m_run));
+          const float p1 = ex2(fmaf(s[c * 32 + 2 * j + 1], sl2, -m_run));
+          sum += p0 + p1;
+          pk[j] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_col + c * 16, pk);
+      }
+      // O of this group is quiescent here (its last P V completed before this S
+      // was signalled), and the next P V is issued only after p_full.
+      if (rescale) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(o_col + c * 32, ov);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+          tmem_st32(o_col + c * 32, ov);
+        }
+      }
+      l_run += sum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl->p_full[x]));
+    }
+    // the group's last P V has completed once its S barrier fires one more time
+    if (ok && n_x > 0) ok = wait_bar_warp(smem_u32(&ctl->s_full[x]), n_x & 1, guard, 7);
+    tc_fence_after();
+    ctl->ml[x][row] = make_float2(n_x > 0 ? m_run : -INFINITY, n_x > 0 ? l_run : 0.f);
+    tc_fence_before();
+    mbar_arrive(smem_u32(&ctl->merge));
+    if (!wait_bar(smem_u32(&ctl->merge), 0, guard, 8)) ok = false;
+    tc_fence_after();
+    const bool go = __all_sync(0xffffffffu, ok && !ctl->abort);
+    if (cnt > 0 && go && row < BN) {
+      const float2 a = ctl->ml[0][row], b = ctl->ml[1][row];
+      const float mm = fmaxf(a.x, b.x);
+      const float fa = a.y > 0.f ? ex2(a.x - mm) : 0.f;
+      const float fb = b.y > 0.f ? ex2(b.x - mm) : 0.f;
+      const float denom = a.y * fa + b.y * fb;
+      const float inv = denom > 0.f ? 1.0f / denom : 0.f;
+      const float ca = fa * inv, cb = fb * inv;
+      __nv_bfloat16* dst = o + ((static_cast<long long>(I) * BN + row) * H + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = x * (D / 2) + c * 32;
+        uint32_t va[32], vb[32];
+        tmem_ld32(tm + lane_off + 256 + col, va);
+        if (n_b > 0) {
+          tmem_ld32(tm + lane_off + 384 + col, vb);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) vb[j] = 0u;
+        }
+        uint4 pk[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float o0 = __uint_as_float(va[2 * j]) * ca + __uint_as_float(vb[2 * j]) * cb;
+          const float o1 = __uint_as_float(va[2 * j + 1]) * ca + __uint_as_float(vb[2 * j + 1]) * cb;
+          pw[j] = pack_bf16x2(o0, o1);
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst + col);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) d4[j] = pk[j];
+      }
+    } else if (cnt == 0 && row < BN) {
+      // no block selected (not a mask rr_search produces): the row has no keys
+      __nv_bfloat16* dst = o + ((static_cast<long long>(I) * BN + row) * H + h) * D;
+      for (int c = x * (D / 2); c < (x + 1) * (D / 2); c += 8)
+        *reinterpret_cast<uint4*>(dst + c) = make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tm, 512);
+}
+
+template <int BN, int D>
+cudaError_t launch_bsfa_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const int32_t* count, const int32_t* idx, void* o, int H, int Hkv, int Nb, float sl2,
+                          const DeviceGuardArgs& g, cudaStream_t stream) {
+  using C = FaCfg<BN, D>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(bsfa_kernel<BN, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  bsfa_kernel<BN, D><<<static_cast<unsigned>(H) * Nb, kThreads, C::kSmem, stream>>>(
+      mq, mk, mv, count, idx, static_cast<__nv_bfloat16*>(o), H, Hkv, Nb, sl2, g.status, g.limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bsfa(const void* q, const void* k, const void* v, const int32_t* count, const int32_t* idx,
+                        void* o, int L, int H, int Hkv, int d, int B, const DeviceGuardArgs& g,
+                        cudaStream_t stream) {
+  const int Nb = L / B;
+  CUtensorMap mq, mk, mv;
+  if (!make_tmap_rows(&mq, q, L, H, d, 128) || !make_tmap_rows(&mk, k, L, Hkv, d, B) ||
+      !make_tmap_rows(&mv, v, L, Hkv, d, B))
+    return cudaErrorInvalidValue;
+  const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
+  if (B == 128 && d == 128) return launch_bsfa_t<128, 128>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, stream);
+  if (B == 128 && d == 64) return launch_bsfa_t<128, 64>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, stream);
+  if (B == 64 && d == 128) return launch_bsfa_t<64, 128>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, stream);
+  if (B == 64 && d == 64) return launch_bsfa_t<64, 64>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rr

@@ -1,0 +1,153 @@
+// rr_abi.cu — the C ABI declared in include/rr.h: host-side validation,
+// workspace carving and stream-ordered launches.  No device memory is
+// allocated here; every buffer is the caller's.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rr.h"
+#include "rr_internal.h"
+
+namespace {
+
+uint64_t g_wait_limit_ns = 2000000000ull;
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  size_t status, khi, klo, mass, total;
+};
+
+Layout carve(int L, int H, int Hkv, int d, int B, int S) {
+  Layout w;
+  const size_t Ns = static_cast<size_t>(L / S), Nb = static_cast<size_t>(L / B);
+  const size_t kbar = round_up(Ns * Hkv * d * 2);
+  w.status = 0;
+  w.khi = kAlign;
+  w.klo = w.khi + kbar;
+  w.mass = w.klo + kbar;
+  w.total = w.mass + round_up(static_cast<size_t>(H) * Nb * Nb * 4);
+  return w;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+rr_status check_shape(int L, int H, int Hkv, int d, int B, int S, bool need_s) {
+  if (L <= 0 || H <= 0 || Hkv <= 0 || d <= 0 || B <= 0) return RR_EINVAL;
+  if (H % Hkv != 0) return RR_EINVAL;
+  if (L % B != 0) return RR_EINVAL;
+  if (need_s && (S <= 0 || B % S != 0)) return RR_EINVAL;
+  if (d != 64 && d != 128) return RR_EUNSUPPORTED;
+  if (B != 64 && B != 128) return RR_EUNSUPPORTED;
+  if (L / B > rr::kMaxBlocks) return RR_EUNSUPPORTED;
+  if (static_cast<long long>(L) * H * d >= (1ll << 40)) return RR_EUNSUPPORTED;
+  return RR_OK;
+}
+
+rr_status check_ws(void* ws, size_t ws_bytes, const Layout& w) {
+  if (!ws) return RR_EINVAL;
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return RR_EALIGN;
+  if (ws_bytes < w.total) return RR_EINVAL;
+  return RR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+rr_status rr_workspace_size(int L, int H, int Hkv, int d, int B, int S, size_t* bytes) {
+  if (!bytes) return RR_EINVAL;
+  rr_status st = check_shape(L, H, Hkv, d, B, S, true);
+  if (st != RR_OK) return st;
+  *bytes = carve(L, H, Hkv, d, B, S).total;
+  return RR_OK;
+}
+
+rr_status rr_search(const void* q, const void* k, int L, int H, int Hkv, int d, int B, int S, float tau,
+                    int32_t* count, int32_t* idx, float* mass, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  rr_status st = check_shape(L, H, Hkv, d, B, S, true);
+  if (st != RR_OK) return st;
+  if (!(tau > 0.0f) || tau != tau) return RR_EINVAL;
+  if (!q || !k || !count || !idx) return RR_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(count) || !aligned16(idx) || (mass && !aligned16(mass)))
+    return RR_EALIGN;
+  const Layout w = carve(L, H, Hkv, d, B, S);
+  if ((st = check_ws(workspace, workspace_bytes, w)) != RR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned int* status = reinterpret_cast<unsigned int*>(ws + w.status);
+  float* m = mass ? mass : reinterpret_cast<float*>(ws + w.mass);
+  const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned int), s) != cudaSuccess) return RR_ECUDA;
+  if (rr::launch_pool_keys(k, ws + w.khi, ws + w.klo, L, Hkv, d, S, s) != cudaSuccess) return RR_ECUDA;
+  if (rr::launch_search(q, ws + w.khi, ws + w.klo, m, L, H, Hkv, d, B, S, g, s) != cudaSuccess) return RR_ECUDA;
+  if (rr::launch_top_tau(m, H, L / B, tau, count, idx, s) != cudaSuccess) return RR_ECUDA;
+  return RR_OK;
+}
+
+rr_status rr_sparse_attn(const void* q, const void* k, const void* v, int L, int H, int Hkv, int d, int B,
+                         const int32_t* count, const int32_t* idx, void* o, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  rr_status st = check_shape(L, H, Hkv, d, B, 1, false);
+  if (st != RR_OK) return st;
+  if (!q || !k || !v || !count || !idx || !o || !workspace) return RR_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(count) || !aligned16(idx))
+    return RR_EALIGN;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return RR_EALIGN;
+  if (workspace_bytes < kAlign) return RR_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int* status = static_cast<unsigned int*>(workspace);
+  const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned int), s) != cudaSuccess) return RR_ECUDA;
+  if (rr::launch_bsfa(q, k, v, count, idx, o, L, H, Hkv, d, B, g, s) != cudaSuccess) return RR_ECUDA;
+  return RR_OK;
+}
+
+rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H, int Hkv, int d, int B, int S,
+                       float tau, int32_t* count, int32_t* idx, void* o, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  rr_status st = check_shape(L, H, Hkv, d, B, S, true);
+  if (st != RR_OK) return st;
+  if (!v || !o) return RR_EINVAL;
+  if (!aligned16(v) || !aligned16(o)) return RR_EALIGN;
+  st = rr_search(q, k, L, H, Hkv, d, B, S, tau, count, idx, nullptr, workspace, workspace_bytes, stream);
+  if (st != RR_OK) return st;
+  // the search's status word stays in place: attention does not reset it
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int* status = static_cast<unsigned int*>(workspace);
+  const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
+  if (rr::launch_bsfa(q, k, v, count, idx, o, L, H, Hkv, d, B, g, s) != cudaSuccess) return RR_ECUDA;
+  return RR_OK;
+}
+
+rr_status rr_check_status(void* workspace, void* stream) {
+  if (!workspace) return RR_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int host = 0;
+  if (cudaMemcpyAsync(&host, workspace, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return RR_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RR_ECUDA;
+  if ((host & 0xFFu) == rr::kStatusTimeoutCode) return RR_ETIMEOUT;
+  return host == 0 ? RR_OK : RR_ECUDA;
+}
+
+uint64_t rr_set_wait_limit_ns(uint64_t ns) {
+  const uint64_t prev = g_wait_limit_ns;
+  g_wait_limit_ns = ns;
+  return prev;
+}
+
+const char* rr_status_string(rr_status s) {
+  switch (s) {
+    case RR_OK: return "ok";
+    case RR_EINVAL: return "invalid argument";
+    case RR_EUNSUPPORTED: return "unsupported shape (d and B must be 64 or 128, L/B <= 4096)";
+    case RR_EALIGN: return "misaligned pointer (16 bytes; workspace 256 bytes)";
+    case RR_ECUDA: return "CUDA error";
+    case RR_ETIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

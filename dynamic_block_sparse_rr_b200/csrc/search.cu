@@ -1,0 +1,319 @@
+// search.cu — the round-robin sampled-score pass and block-mass aggregation
+// (RRAttention abstract: "head round-robin (RR) sampling", "stride-level
+// aggregation", "O(L^2/S^2)"; Figure 2 stages 1 and 2).
+//
+// Head h samples, in stride i, the query at position i*S + (h mod S).  These
+// Ns = L/S real queries are scored against the Ns stride-pooled keys of the
+// head's kv group: s[i, j] = q_i . kbar_j / sqrt(d) for j <= i.  That is a
+// causal "mini attention" of length Ns, computed in 128 x 128 tiles:
+//
+//   * one CTA per (head, tile of 128 sampled rows); heavier tiles launch first;
+//   * the sampled rows are read zero-copy through a 4D TMA view of q
+//     (d, H, S, Ns), so no sampled copy is ever materialised;
+//   * S = Qs Kbar^T runs on tcgen05 (bf16 in, fp32 accumulate in TMEM) as two
+//     MMA chains, Qs*Khi^T + Qs*Klo^T, so the pooled keys enter at ~16 bits;
+//   * pass 1 walks the row's key tiles for the row log-sum-exp (online), pass 2
+//     recomputes the identical scores, forms P = exp(s - lse) and sums P over
+//     the r x r (sampled row, stride) pairs of each B x B block with warp
+//     shuffles; the block masses go to global memory.
+//
+// Warp roles: warp 0 issues TMA, warp 1 issues MMAs (one thread) and owns the
+// TMEM allocation, warps 2..5 (128 threads, thread = sampled row = TMEM lane)
+// do the softmax and reductions.  TMEM: two 128-column fp32 score buffers, so
+// the MMA of tile n+1 overlaps the softmax of tile n.  Small shared memory
+// lets two CTAs share an SM, whose tensor core then alternates between them.
+#include <cuda_bf16.h>
+
+#include "rr_internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace rr {
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kThreads = 192;
+
+template <int D>
+struct SearchCfg {
+  static constexpr int kStages = D == 128 ? 2 : 4;       // pooled-key tiles (hi or lo) in flight
+  static constexpr int kTileBytes = kTile * D * 2;       // one 128 x D bf16 tile
+  static constexpr int kQOff = 0;
+  static constexpr int kStageOff = kTileBytes;
+  static constexpr int kCtrlOff = kStageOff + kStages * kTileBytes;
+  static constexpr int kSmem = kCtrlOff + 1024 + 1024;   // control block + alignment slack
+};
+
+struct SearchCtrl {
+  uint64_t full[4];
+  uint64_t empty[4];
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t s_empty[2];
+  uint64_t drain;
+  uint64_t red_bar;   // the 128 reduction threads meet here (bounded, unlike bar.sync)
+  uint32_t tmem_base;
+  int abort;
+  float red[4][4];   // cross-warp partial block sums when r > 32
+};
+
+template <int D, int LOGR>
+__global__ void __launch_bounds__(kThreads, 2)
+    search_kernel(const __grid_constant__ CUtensorMap mqs, const __grid_constant__ CUtensorMap mkh,
+                  const __grid_constant__ CUtensorMap mkl, float* __restrict__ mass, int H, int Hkv, int S,
+                  int Ns, int Nb, float sl2, unsigned int* status, uint64_t limit_ns) {
+  using C = SearchCfg<D>;
+  constexpr int R = 1 << LOGR;                 // sampled rows (and strides) per block
+  constexpr int GPT = kTile / R;               // key blocks per 128-stride tile
+  constexpr int KSTEPS = D / 16;
+  constexpr uint32_t kIdesc = idesc_bf16_f32(128, kTile, false, false);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::kQOff;
+  uint8_t* sStage = smem + C::kStageOff;
+  SearchCtrl* ctl = reinterpret_cast<SearchCtrl*>(smem + C::kCtrlOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_row_tiles = (Ns + kTile - 1) / kTile;
+  const int rt = n_row_tiles - 1 - static_cast<int>(blockIdx.x / H);   // row tile, heavy first
+  const int h = static_cast<int>(blockIdx.x % H);
+  const int kvh = h / (H / Hkv);
+  const int n_key_tiles = rt + 1;
+  const int n_seq = 2 * n_key_tiles;           // pass 1 then pass 2
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 1);
+    }
+    mbar_init(smem_u32(&ctl->q_full), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ctl->s_full[b]), 1);
+      mbar_init(smem_u32(&ctl->s_empty[b]), 128);
+    }
+    mbar_init(smem_u32(&ctl->drain), 1);
+    mbar_init(smem_u32(&ctl->red_bar), 128);
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = ctl->tmem_base;
+  const Guard guard{&ctl->abort, status, limit_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&mqs);
+      tma_prefetch_desc(&mkh);
+      tma_prefetch_desc(&mkl);
+      const uint32_t qb = smem_u32(&ctl->q_full);
+      mbar_expect_tx(qb, C::kTileBytes);
+      for (int a = 0; a < D / 64; ++a)
+        tma_load_4d(smem_u32(sQ + a * kTile * 128), &mqs, qb, a * 64, h, h % S, rt * kTile);
+      int k = 0;
+      bool ok = true;
+      for (int n = 0; n < n_seq && ok; ++n) {
+        const int c = n % n_key_tiles;
+        for (int part = 0; part < 2 && ok; ++part) {
+          const int st = k % C::kStages;
+          const uint32_t ph = (k / C::kStages) & 1;
+          if (!wait_bar(smem_u32(&ctl->empty[st]), ph ^ 1, guard, 1)) { ok = false; break; }
+          const uint32_t fb = smem_u32(&ctl->full[st]);
+          mbar_expect_tx(fb, C::kTileBytes);
+          uint8_t* dst = sStage + st * C::kTileBytes;
+          for (int a = 0; a < D / 64; ++a)
+            tma_load_3d(smem_u32(dst + a * kTile * 128), part == 0 ? &mkh : &mkl, fb, a * 64, kvh, c * kTile);
+          ++k;
+        }
+      }
+      // drain: every issued load has landed before the CTA may exit
+      drain_bar(qb, 0, kDrainLimitNs);
+      for (int kk = (k > C::kStages ? k - C::kStages : 0); kk < k; ++kk)
+        drain_bar(smem_u32(&ctl->full[kk % C::kStages]), (kk / C::kStages) & 1, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = wait_bar(smem_u32(&ctl->q_full), 0, guard, 2);
+      tc_fence_after();
+      int k = 0;
+      for (int n = 0; n < n_seq && ok; ++n) {
+        const int b = n & 1;
+        if (!wait_bar(smem_u32(&ctl->s_empty[b]), ((n >> 1) & 1) ^ 1, guard, 3)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dcol = tm + b * kTile;
+        for (int part = 0; part < 2; ++part) {
+          const int st = k % C::kStages;
+          if (!wait_bar(smem_u32(&ctl->full[st]), (k / C::kStages) & 1, guard, 4)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* kt = sStage + st * C::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < KSTEPS; ++kk) {
+            const uint64_t ad = sdesc_sw128(smem_u32(sQ + (kk >> 2) * kTile * 128 + 32 * (kk & 3)), 16, 1024);
+            const uint64_t bd = sdesc_sw128(smem_u32(kt + (kk >> 2) * kTile * 128 + 32 * (kk & 3)), 16, 1024);
+            umma_ss(dcol, ad, bd, kIdesc, (part > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&ctl->empty[st]));
+          ++k;
+        }
+        if (!ok) break;
+        umma_commit(smem_u32(&ctl->s_full[b]));
+      }
+      umma_commit(smem_u32(&ctl->drain));
+      drain_bar(smem_u32(&ctl->drain), 0, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax / reduction
+    const int wq = warp & 3;                    // TMEM lane quarter of this warp
+    const int row = wq * 32 + lane;             // sampled row within the tile
+    const int i = rt * kTile + row;             // sampled row index (stride of the query)
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    float m_run = -INFINITY, l_run = 0.f, lse = 0.f;
+    uint32_t red_phase = 0;
+    bool ok = true;
+    for (int n = 0; n < n_seq; ++n) {
+      const int b = n & 1;
+      const int c = n % n_key_tiles;
+      const bool pass2 = n >= n_key_tiles;
+      if (!wait_bar_warp(smem_u32(&ctl->s_full[b]), (n >> 1) & 1, guard, 5)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t raw[128];
+      tmem_ld128(tm + lane_off + b * kTile, raw);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl->s_empty[b]));
+      float v[128];
+      const bool diag = (c == rt);
+#pragma unroll
+      for (int j = 0; j < 128; ++j) {
+        const float x = __uint_as_float(raw[j]) * sl2;
+        v[j] = (diag && j > row) ? -INFINITY : x;   // stride-causal: j <= i
+      }
+      if (!pass2) {
+        float mx = v[0];
+#pragma unroll
+        for (int j = 1; j < 128; ++j) mx = fmaxf(mx, v[j]);
+        const float m_new = fmaxf(m_run, mx);
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 128; ++j) sum += ex2(v[j] - m_new);
+        l_run = l_run * ex2(m_run - m_new) + sum;
+        m_run = m_new;
+        if (n == n_key_tiles - 1) lse = m_run + lg2(l_run);
+        continue;
+      }
+      // pass 2: probabilities, summed over each key block's R strides (in place: v[g])
+#pragma unroll
+      for (int g = 0; g < GPT; ++g) {
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < R; ++t) acc += ex2(v[g * R + t] - lse);
+        v[g] = acc;
+      }
+      // ... and over the R sampled rows of each query block
+      if constexpr (R <= 32) {
+#pragma unroll
+        for (int g = 0; g < GPT; ++g) {
+#pragma unroll
+          for (int off = 1; off < R; off <<= 1) v[g] += __shfl_xor_sync(0xffffffffu, v[g], off);
+        }
+        const int I = i >> LOGR;
+        if ((lane & (R - 1)) == 0 && I < Nb) {
+          float* dst = mass + (static_cast<long long>(h) * Nb + I) * Nb + c * GPT;
+#pragma unroll
+          for (int g = 0; g < GPT; ++g)
+            if (c * GPT + g < Nb) dst[g] = v[g];
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < GPT; ++g) {
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) v[g] += __shfl_xor_sync(0xffffffffu, v[g], off);
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int g = 0; g < GPT; ++g) ctl->red[wq][g] = v[g];
+        }
+        mbar_arrive(smem_u32(&ctl->red_bar));
+        if (!wait_bar_warp(smem_u32(&ctl->red_bar), red_phase++ & 1, guard, 6)) { ok = false; break; }
+        constexpr int WPB = R / 32;             // warps per query block
+        const int t = threadIdx.x - 64;
+        if (t < (4 / WPB) * GPT) {
+          const int qb = t / GPT, g = t % GPT;
+          float acc = 0.f;
+          for (int w = 0; w < WPB; ++w) acc += ctl->red[qb * WPB + w][g];
+          const int I = (rt * kTile) / R + qb;
+          if (I < Nb && c * GPT + g < Nb) mass[(static_cast<long long>(h) * Nb + I) * Nb + c * GPT + g] = acc;
+        }
+        mbar_arrive(smem_u32(&ctl->red_bar));
+        if (!wait_bar_warp(smem_u32(&ctl->red_bar), red_phase++ & 1, guard, 7)) { ok = false; break; }
+      }
+    }
+    (void)ok;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tm, 256);
+}
+
+template <int D, int LOGR>
+cudaError_t launch_search_t(const CUtensorMap& mqs, const CUtensorMap& mkh, const CUtensorMap& mkl, float* mass,
+                            int H, int Hkv, int S, int Ns, int Nb, float sl2, const DeviceGuardArgs& g,
+                            cudaStream_t stream) {
+  using C = SearchCfg<D>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(search_kernel<D, LOGR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int n_row_tiles = (Ns + kTile - 1) / kTile;
+  search_kernel<D, LOGR><<<static_cast<unsigned>(n_row_tiles) * H, kThreads, C::kSmem, stream>>>(
+      mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, g.status, g.limit_ns);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t dispatch_r(int logr, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, float* mass,
+                       int H, int Hkv, int S, int Ns, int Nb, float sl2, const DeviceGuardArgs& g, cudaStream_t st) {
+  switch (logr) {
+    case 0: return launch_search_t<D, 0>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
+    case 1: return launch_search_t<D, 1>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
+    case 2: return launch_search_t<D, 2>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
+    case 3: return launch_search_t<D, 3>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
+    case 4: return launch_search_t<D, 4>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
+    case 5: return launch_search_t<D, 5>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
+    case 6: return launch_search_t<D, 6>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
+    case 7: return launch_search_t<D, 7>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_search(const void* q, const void* khi, const void* klo, float* mass, int L, int H, int Hkv,
+                          int d, int B, int S, const DeviceGuardArgs& g, cudaStream_t stream) {
+  const int Ns = L / S, Nb = L / B, r = B / S;
+  int logr = 0;
+  while ((1 << logr) < r) ++logr;
+  CUtensorMap mqs, mkh, mkl;
+  if (!make_tmap_sampled(&mqs, q, L, H, d, S, kTile) || !make_tmap_rows(&mkh, khi, Ns, Hkv, d, kTile) ||
+      !make_tmap_rows(&mkl, klo, Ns, Hkv, d, kTile))
+    return cudaErrorInvalidValue;
+  const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
+  if (d == 128) return dispatch_r<128>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, g, stream);
+  return dispatch_r<64>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, g, stream);
+}
+
+}  // namespace rr

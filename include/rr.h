@@ -1,0 +1,110 @@
+/*
+ * rr.h — C ABI of the B200 (sm_100a) RRAttention prefill operator.
+ *
+ * The operator is the one described in "RRAttention: Dynamic Block Sparse
+ * Attention via Per-Head Round-Robin Shifts for Long-Context Inference"
+ * (Abstract and TL;DR; Figure 2 caption for the three stages): a head
+ * round-robin strided pattern search that selects, per query block, an
+ * adaptive Top-tau set of key blocks (the last query block kept dense),
+ * followed by causal block-sparse attention over the selected blocks.
+ *
+ * Notation: H query heads, Hkv kv heads (H % Hkv == 0, g = H/Hkv), head dim d,
+ * sequence length L, block size B, stride S; Ns = L/S, Nb = L/B, r = B/S.
+ *
+ * Layouts (row-major, batch 1; a batch is a loop over calls):
+ *   q, o : [L, H, d]   bf16          k, v : [L, Hkv, d] bf16
+ *   count: [H, Nb]     int32         idx  : [H, Nb, Nb] int32
+ * Mask format: count[h*Nb+I] in [1, I+1]; idx[(h*Nb+I)*Nb + t], t < count, lists
+ * the selected key blocks of row I in strictly ascending order (so J = I, when
+ * selected, is last).  Entries at t >= count are not written and not read.
+ *
+ * Ownership: the caller allocates every buffer (device memory unless stated);
+ * the library never allocates or frees device memory.  All device work is
+ * enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and the
+ * calls return without synchronising, except rr_check_status.
+ *
+ * Errors: arguments are validated on the host before anything is enqueued:
+ * RR_EINVAL (sizes, tau, null pointers), RR_EUNSUPPORTED (d or B outside
+ * {64, 128}), RR_EALIGN (a device pointer not 16-byte aligned, or a workspace
+ * not 256-byte aligned), RR_ECUDA (a launch failed).  Device-side failures (a
+ * bounded wait that ran out) are recorded in a status word inside the
+ * workspace; rr_check_status returns them.
+ */
+#ifndef RR_H_
+#define RR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RR_OK = 0,
+  RR_EINVAL = 1,
+  RR_EUNSUPPORTED = 2,
+  RR_EALIGN = 3,
+  RR_ECUDA = 4,
+  RR_ETIMEOUT = 5
+} rr_status;
+
+/* Bytes of device workspace that rr_search / rr_sparse_attn / rr_attention
+ * need for this shape (pooled keys, block masses, status word).  The same
+ * workspace may be reused by consecutive calls on one stream. */
+rr_status rr_workspace_size(int L, int H, int Hkv, int d, int B, int S, size_t* bytes);
+
+/* Pattern search (Abstract: head round-robin sampling, stride-level
+ * aggregation, adaptive Top-tau; TL;DR: static protection of the last query
+ * block; Figure 2 stages 1 and 2).
+ *   Sampling: head h samples, in stride i, the query at i*S + (h mod S).
+ *   Keys:     the S keys of stride j are averaged (fp32, kept as a bf16 pair).
+ *   Scores:   s[h,i,j] = q . kbar[j] / sqrt(d) for j <= i, softmax per row.
+ *   Mass:     summed over the r x r (row, stride) pairs of block (I, J).
+ *   Top-tau:  per row I < Nb-1, blocks in (mass desc, J asc) order, shortest
+ *             prefix whose share of the row's mass is >= tau (tau >= 1: all).
+ *             Row Nb-1 keeps all blocks.
+ * In:  q [L,H,d], k [L,Hkv,d] bf16 (device); tau > 0.
+ * Out: count [H,Nb], idx [H,Nb,Nb] int32 (device, caller-owned).
+ *      mass: NULL, or a device [H,Nb,Nb] fp32 buffer that receives the
+ *      unnormalised block mass (entries J <= I; others unspecified).
+ * Requires L % B == 0, B % S == 0, d and B in {64, 128}. */
+rr_status rr_search(const void* q, const void* k, int L, int H, int Hkv, int d, int B, int S,
+                    float tau, int32_t* count, int32_t* idx, float* mass, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Causal block-sparse attention over a block mask (Abstract: "computing only
+ * half of the attention blocks"; Figure 2 stage 3).  Query q of block I, head
+ * h, attends with scale 1/sqrt(d) to every key k <= q of the blocks listed for
+ * (h, I); kv head = h / (H/Hkv).  fp32 softmax and accumulation, bf16 output.
+ * In:  q, k, v bf16 (device), count/idx as produced by rr_search (any valid
+ *      mask in the format above is accepted; entries are not range-checked on
+ *      the device beyond the debug checks of the kernel).
+ * Out: o [L,H,d] bf16 (device, caller-owned). */
+rr_status rr_sparse_attn(const void* q, const void* k, const void* v, int L, int H, int Hkv, int d,
+                         int B, const int32_t* count, const int32_t* idx, void* o, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* rr_search followed by rr_sparse_attn on the same stream.  count/idx are
+ * caller-provided device buffers that receive the mask. */
+rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H, int Hkv, int d,
+                       int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, returns the device-side status recorded since the
+ * last rr_* call that started on this workspace (RR_OK or RR_ETIMEOUT), and
+ * RR_ECUDA if the stream reports an error. */
+rr_status rr_check_status(void* workspace, void* stream);
+
+/* Sets the bound, in nanoseconds, of every device-side wait of later launches
+ * (default 2e9).  Returns the previous bound.  Process-wide. */
+uint64_t rr_set_wait_limit_ns(uint64_t ns);
+
+/* Static string for a status code. */
+const char* rr_status_string(rr_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RR_H_ */

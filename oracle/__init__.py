@@ -52,7 +52,8 @@ B=8); R6 against brute-force subset enumeration; R7 by inspection of every row.
 R2 and R3 for S > 1 have no pin beyond those reductions: "parity unpinned".
 
 All arithmetic is float64.  Inputs are the bf16 values both paths receive,
-widened exactly.
+widened exactly (callers may pass them as float32 or float64 arrays; every
+function widens to float64 before any arithmetic).
 """
 from __future__ import annotations
 
@@ -73,7 +74,7 @@ def sampled_positions(L: int, H: int, S: int) -> np.ndarray:
 def pool_keys(K: np.ndarray, S: int) -> np.ndarray:
     """Kbar[j, kv, :] = mean over the S keys of stride j (R2).  K: [L, Hkv, d]."""
     L, Hkv, d = K.shape
-    return K.reshape(L // S, S, Hkv, d).mean(axis=1)
+    return K.astype(np.float64).reshape(L // S, S, Hkv, d).mean(axis=1)
 
 
 # ------------------------------------------------------- R3-R5 block masses
@@ -92,7 +93,7 @@ def block_mass(Q: np.ndarray, K: np.ndarray, B: int, S: int, row_chunk: int = 20
     M = np.zeros((H, Nb, Nb), dtype=np.float64)
     step = max(r, (row_chunk // r) * r)
     for h in range(H):
-        Qs = Q[pos[h], h, :]                     # [Ns, d] real sampled queries
+        Qs = Q[pos[h], h, :].astype(np.float64)  # [Ns, d] real sampled queries
         Kb = Kbar[:, h // g, :]                  # [Ns, d]
         for a in range(0, Ns, step):
             b = min(Ns, a + step)
@@ -175,12 +176,12 @@ def sparse_attention_block(Q, K, V, h: int, I: int, blocks, B: int) -> np.ndarra
     blocks = np.asarray(blocks, dtype=np.int64)
     keys = (blocks[:, None] * B + np.arange(B)[None, :]).reshape(-1)
     q_pos = I * B + np.arange(B)
-    s = (Q[q_pos, h, :] @ K[keys, kv, :].T) / math.sqrt(d)
+    s = (Q[q_pos, h, :].astype(np.float64) @ K[keys, kv, :].astype(np.float64).T) / math.sqrt(d)
     s = np.where(keys[None, :] <= q_pos[:, None], s, -np.inf)
     s = s - s.max(axis=1, keepdims=True)
     p = np.exp(s)
     p = p / p.sum(axis=1, keepdims=True)
-    return p @ V[keys, kv, :]
+    return p @ V[keys, kv, :].astype(np.float64)
 
 
 def sparse_attention(Q, K, V, count, idx, B: int, rows=None) -> np.ndarray:

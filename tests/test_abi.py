@@ -1,0 +1,121 @@
+"""The C ABI: the library loads, exports every symbol rr.h declares, and rejects
+bad arguments on the host (no GPU needed; no compute call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rr.h")
+
+
+@pytest.fixture(scope="module")
+def rr():
+    from dynamic_block_sparse_rr_b200 import _build
+    _build.build()
+    import dynamic_block_sparse_rr_b200 as m
+    m.lib()
+    return m
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rr_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(rr):
+    names = _declared()
+    assert names == sorted(rr.EXPORTS)
+    for n in names:
+        assert hasattr(rr.lib(), n), n
+
+
+def test_status_strings(rr):
+    for code in range(6):
+        s = rr.status_string(code)
+        assert isinstance(s, str) and s
+    assert rr.status_string(0) == "ok"
+
+
+def test_wait_limit_roundtrip(rr):
+    prev = rr.set_wait_limit_ns(12345)
+    assert rr.set_wait_limit_ns(prev) == 12345
+
+
+def _ws(L, H, Hkv, d, B, S):
+    n = ctypes.c_size_t()
+    code = rr_lib().rr_workspace_size(L, H, Hkv, d, B, S, ctypes.byref(n))
+    return code, n.value
+
+
+def rr_lib():
+    import dynamic_block_sparse_rr_b200 as m
+    return m.lib()
+
+
+@pytest.mark.parametrize("args,code", [
+    ((1024, 4, 4, 64, 64, 4), 0),
+    ((131072, 32, 8, 128, 128, 16), 0),
+    ((1024, 4, 3, 64, 64, 4), 1),      # H % Hkv
+    ((1000, 4, 4, 64, 64, 4), 1),      # L % B
+    ((1024, 4, 4, 64, 64, 3), 1),      # B % S
+    ((1024, 4, 4, 64, 64, 0), 1),
+    ((1024, 4, 4, 96, 64, 4), 2),      # d
+    ((1024, 4, 4, 64, 32, 4), 2),      # B
+    ((64 * 8192, 1, 1, 64, 64, 4), 2),  # Nb > 4096
+    ((0, 4, 4, 64, 64, 4), 1),
+])
+def test_workspace_size_validation(rr, args, code):
+    c, n = _ws(*args)
+    assert c == code
+    if code == 0:
+        L, H, Hkv, d, B, S = args
+        assert n >= H * (L // B) ** 2 * 4 + 2 * (L // S) * Hkv * d * 2
+
+
+def test_search_rejects_before_any_launch(rr):
+    lib = rr.lib()
+    good = 1 << 20            # fake, 16-byte aligned "device" addresses: never dereferenced
+    L, H, Hkv, d, B, S = 1024, 4, 4, 64, 64, 4
+    _, n = _ws(L, H, Hkv, d, B, S)
+    args = dict(q=good, k=good, tau=0.9, count=good, idx=good, mass=None, ws=good, nws=n)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.rr_search(a["q"], a["k"], L, H, Hkv, d, B, S, a["tau"], a["count"], a["idx"], a["mass"],
+                             a["ws"], a["nws"], None)
+
+    assert call(q=None) == rr.RR_EINVAL
+    assert call(idx=None) == rr.RR_EINVAL
+    assert call(tau=0.0) == rr.RR_EINVAL
+    assert call(tau=-1.0) == rr.RR_EINVAL
+    assert call(tau=float("nan")) == rr.RR_EINVAL
+    assert call(q=good + 8) == rr.RR_EALIGN
+    assert call(mass=good + 4) == rr.RR_EALIGN
+    assert call(ws=good + 16) == rr.RR_EALIGN
+    assert call(nws=n - 1) == rr.RR_EINVAL
+    assert call(ws=None) == rr.RR_EINVAL
+    assert lib.rr_search(good, good, L, H, Hkv, d, 32, S, 0.9, good, good, None, good, n, None) == rr.RR_EUNSUPPORTED
+
+
+def test_sparse_attn_and_attention_reject(rr):
+    lib = rr.lib()
+    g = 1 << 20
+    L, H, Hkv, d, B = 1024, 4, 2, 128, 128
+    assert lib.rr_sparse_attn(g, g, g, L, H, Hkv, d, B, g, g, None, g, 256, None) == rr.RR_EINVAL
+    assert lib.rr_sparse_attn(g, g, g + 2, L, H, Hkv, d, B, g, g, g, g, 256, None) == rr.RR_EALIGN
+    assert lib.rr_sparse_attn(g, g, g, L, H, Hkv, d, B, g, g, g, g + 64, 256, None) == rr.RR_EALIGN
+    assert lib.rr_sparse_attn(g, g, g, L, H, 3, d, B, g, g, g, g, 256, None) == rr.RR_EINVAL
+    assert lib.rr_sparse_attn(g, g, g, L, H, Hkv, 80, B, g, g, g, g, 256, None) == rr.RR_EUNSUPPORTED
+    assert lib.rr_attention(g, g, None, L, H, Hkv, d, B, 16, 0.95, g, g, g, g, 1 << 30, None) == rr.RR_EINVAL
+    assert lib.rr_attention(g, g, g, L, H, Hkv, d, B, 16, 0.0, g, g, g, g, 1 << 30, None) == rr.RR_EINVAL
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    import dynamic_block_sparse_rr_b200 as m
+    monkeypatch.setattr(m, "LIB_PATH", os.path.join(ROOT, "no", "such", "librr.so"))
+    monkeypatch.setattr(m, "_lib", None)
+    with pytest.raises(ImportError):
+        m.lib()

@@ -1,0 +1,239 @@
+"""CUDA path vs the fp64 oracle, through the C ABI.
+
+Masks: bit-exact except blocks in the 1e-4 band around tau (or near-ties at the
+cut), which are counted and reported.  Outputs (bf16) against the oracle fed
+the GPU's own mask: max |err| <= 2e-2, mean |err| <= 2e-3.  Block masses are
+also compared directly (normalised, |err| <= 2e-5): they are fp32 on the GPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gen
+import oracle
+from tests.mask_compare import check_mask_format, compare_masks, output_errors
+
+pytestmark = pytest.mark.gpu
+
+MAX_ERR, MEAN_ERR, MASS_ERR = 2e-2, 2e-3, 2e-5
+
+
+@pytest.fixture(scope="module")
+def rr():
+    from dynamic_block_sparse_rr_b200 import _build
+    _build.build()
+    import dynamic_block_sparse_rr_b200 as m
+    assert torch.cuda.is_available(), "the parity tests need a CUDA device"
+    m.lib()
+    return m
+
+
+def to_dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def run_gpu(rr, qd, kd, vd, B, S, tau):
+    L, H, d = qd.shape
+    Hkv = kd.shape[1]
+    Nb = L // B
+    ws = rr.workspace(L, H, Hkv, d, B, S)
+    mass = torch.zeros((H, Nb, Nb), dtype=torch.float32, device="cuda")
+    count, idx = rr.search(qd, kd, B, S, tau, mass=mass, ws=ws)
+    o = rr.sparse_attn(qd, kd, vd, count, idx, B, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+    torch.cuda.synchronize()
+    return count.cpu().numpy(), idx.cpu().numpy(), mass.cpu().numpy().astype(np.float64), o
+
+
+def gpu_o_f32(o: torch.Tensor) -> np.ndarray:
+    return o.float().cpu().numpy()
+
+
+def normalised(M):
+    return oracle.normalise_mass(M)
+
+
+def check_case(rr, L, H, Hkv, d, B, S, tau, structure, seed=0, attn_rows=None, taus=None):
+    q, k, v = gen.make_qkv(L, H, Hkv, d, structure, seed)
+    Q, K, V = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k), gen.bf16_bits_to_f32(v)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    Nb = L // B
+    M_o = oracle.block_mass(Q, K, B, S)
+    m_o = normalised(M_o)
+    report = {}
+    for t in (taus or [tau]):
+        count, idx, M_g, o = run_gpu(rr, qd, kd, vd, B, S, t)
+        check_mask_format(count, idx)
+        tri = np.tri(Nb, dtype=bool)[None]
+        mass_err = float(np.max(np.abs(np.where(tri, normalised(M_g) - m_o, 0.0))))
+        assert mass_err <= MASS_ERR, f"block mass error {mass_err}"
+        count_o, idx_o = oracle.select(m_o, t)
+        st = compare_masks(count, idx, count_o, idx_o, m_o, t)
+        assert st["blocks_fail"] == 0, st
+        O_ref = oracle.sparse_attention(Q, K, V, count, idx, B, rows=attn_rows)
+        mx, mean = output_errors(gpu_o_f32(o), O_ref)
+        assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
+        report[t] = dict(mass_err=mass_err, max_err=mx, mean_err=mean,
+                         visited=float(count.sum()) / (H * Nb * (Nb + 1) / 2), **st)
+    print(report)
+    return report
+
+
+# ------------------------------------------------------------ small, full check
+def test_tiny_config(rr):
+    cfg = gen.CONFIGS["tiny"]
+    check_case(rr, cfg.L, cfg.H, cfg.Hkv, cfg.d, cfg.B, cfg.S, cfg.tau, cfg.structure)
+
+
+@pytest.mark.parametrize("L,H,Hkv,d,B,S,tau,structure", [
+    (1600, 4, 2, 64, 64, 4, 0.9, gen.PLANTED),        # Ns = 400: ragged sampled-row tile
+    (4096, 8, 2, 128, 128, 16, 0.95, gen.PLANTED),   # LLaMA-shaped head dim / block
+    (2240, 4, 1, 128, 64, 8, 0.9, gen.PLANTED_BAND),  # B=64 with d=128, Nb = 35
+    (2048, 2, 2, 64, 128, 2, 0.8, gen.IID),          # r = 64: cross-warp block reduction
+    (1024, 2, 1, 128, 128, 1, 0.9, gen.PLANTED),     # S = 1: every query sampled, r = 128
+    (4096, 7, 1, 128, 128, 16, 0.95, gen.VIDEO),     # video-like frames, GQA 7:1
+    (512, 3, 3, 64, 64, 64, 0.5, gen.IID),           # r = 1
+])
+def test_small_shapes(rr, L, H, Hkv, d, B, S, tau, structure):
+    check_case(rr, L, H, Hkv, d, B, S, tau, structure, seed=1)
+
+
+@pytest.mark.parametrize("B,d", [(64, 64), (128, 128)])
+def test_single_block_and_two_blocks(rr, B, d):
+    for L in (B, 2 * B):
+        check_case(rr, L, 2, 1, d, B, 4, 0.9, gen.IID, seed=2)
+
+
+@pytest.mark.parametrize("B,d", [(64, 64), (64, 128), (128, 64), (128, 128)])
+def test_tau_one_is_dense_causal(rr, B, d):
+    L, H, Hkv = 8 * B, 4, 2
+    q, k, v = gen.make_qkv(L, H, Hkv, d, gen.IID, 3)
+    Q, K, V = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k), gen.bf16_bits_to_f32(v)
+    count, idx, _, o = run_gpu(rr, to_dev(q), to_dev(k), to_dev(v), B, 4, 1.0)
+    c_ref, i_ref = oracle.full_causal_mask(H, L // B)
+    assert np.array_equal(count, c_ref)
+    for h in range(H):
+        for I in range(L // B):
+            assert np.array_equal(idx[h, I, :count[h, I]], i_ref[h, I, :count[h, I]])
+    O_ref = oracle.sparse_attention(Q, K, V, c_ref, i_ref, B)
+    mx, mean = output_errors(gpu_o_f32(o), O_ref)
+    assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
+
+
+@pytest.mark.parametrize("B,d", [(64, 64), (128, 128), (64, 128)])
+def test_arbitrary_masks(rr, B, d):
+    """Attention over masks not produced by the search: single blocks, diagonal
+    only, gaps, long lists."""
+    L, H, Hkv = 12 * B, 4, 2
+    Nb = L // B
+    rng = np.random.default_rng(7)
+    q, k, v = gen.make_qkv(L, H, Hkv, d, gen.IID, 4)
+    Q, K, V = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k), gen.bf16_bits_to_f32(v)
+    count = np.zeros((H, Nb), np.int32)
+    idx = np.zeros((H, Nb, Nb), np.int32)
+    for h in range(H):
+        for I in range(Nb):
+            kind = (h + I) % 4
+            if kind == 0:
+                sel = np.array([I])
+            elif kind == 1:
+                sel = np.array([rng.integers(0, I + 1)])
+            elif kind == 2:
+                sel = np.arange(I + 1)
+            else:
+                sel = np.nonzero(rng.random(I + 1) < 0.4)[0]
+                if sel.size == 0:
+                    sel = np.array([0])
+            count[h, I] = sel.size
+            idx[h, I, :sel.size] = sel
+    cd, idd = torch.from_numpy(count).cuda(), torch.from_numpy(idx).cuda()
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    o = rr.sparse_attn(qd, kd, vd, cd, idd, B, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+    O_ref = oracle.sparse_attention(Q, K, V, count, idx, B)
+    mx, mean = output_errors(gpu_o_f32(o), O_ref)
+    assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
+
+
+def test_deterministic(rr):
+    L, H, Hkv, d, B, S = 4096, 8, 2, 128, 128, 16
+    q, k, v = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 5)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    a = run_gpu(rr, qd, kd, vd, B, S, 0.95)
+    b = run_gpu(rr, qd, kd, vd, B, S, 0.95)
+    assert np.array_equal(a[0], b[0])
+    for h in range(H):
+        for I in range(L // B):
+            assert np.array_equal(a[1][h, I, :a[0][h, I]], b[1][h, I, :b[0][h, I]])
+    assert np.array_equal(a[2], b[2])
+    assert torch.equal(a[3], b[3])
+
+
+def test_fused_attention_matches_two_calls(rr):
+    L, H, Hkv, d, B, S = 2048, 4, 2, 128, 128, 16
+    q, k, v = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 6)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    c1, i1, _, o1 = run_gpu(rr, qd, kd, vd, B, S, 0.9)
+    ws = rr.workspace(L, H, Hkv, d, B, S)
+    o2, c2, i2 = rr.attention(qd, kd, vd, B, S, 0.9, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+    assert np.array_equal(c1, c2.cpu().numpy())
+    assert torch.equal(o1, o2)
+
+
+# ------------------------------------------------------------ full-size workloads
+def _sampled_rows(count, H, Nb, seed, n_random=24):
+    rng = np.random.default_rng(seed)
+    rows = {(h, 0) for h in (0, H - 1)} | {(h, Nb - 1) for h in (0, H // 2, H - 1)}
+    heavy = np.argsort(-count.reshape(-1))[:4]
+    rows |= {(int(i // Nb), int(i % Nb)) for i in heavy}
+    rows |= {(int(rng.integers(0, H)), int(rng.integers(0, Nb))) for _ in range(n_random)}
+    return sorted(rows)
+
+
+def check_full_config(rr, name, taus=None):
+    cfg = gen.CONFIGS[name]
+    q, k, v = gen.make_config(cfg)
+    Q, K, V = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k), gen.bf16_bits_to_f32(v)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    Nb = cfg.L // cfg.B
+    m_o = oracle.normalise_mass(oracle.block_mass(Q, K, cfg.B, cfg.S))
+    out = {}
+    for t in (taus or [cfg.tau]):
+        count, idx, M_g, o = run_gpu(rr, qd, kd, vd, cfg.B, cfg.S, t)
+        check_mask_format(count, idx)
+        tri = np.tri(Nb, dtype=bool)[None]
+        mass_err = float(np.max(np.abs(np.where(tri, oracle.normalise_mass(M_g) - m_o, 0.0))))
+        assert mass_err <= MASS_ERR, mass_err
+        count_o, idx_o = oracle.select(m_o, t)
+        st = compare_masks(count, idx, count_o, idx_o, m_o, t)
+        assert st["blocks_fail"] == 0, st
+        rows = _sampled_rows(count, cfg.H, Nb, 11)
+        O_ref = oracle.sparse_attention(Q, K, V, count, idx, cfg.B, rows=rows)
+        mx, mean = output_errors(gpu_o_f32(o), O_ref)
+        assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
+        out[t] = dict(mass_err=mass_err, max_err=mx, mean_err=mean, rows_checked=len(rows),
+                      visited=float(count.sum()) / (cfg.H * Nb * (Nb + 1) / 2), **st)
+    print(name, out)
+    return out
+
+
+@pytest.mark.slow
+def test_llama16k(rr):
+    check_full_config(rr, "llama16k")
+
+
+@pytest.mark.slow
+def test_llama32k_tau_sweep(rr):
+    check_full_config(rr, "llama32k", taus=[0.9, 0.95, 0.99])
+
+
+@pytest.mark.slow
+def test_video64k(rr):
+    check_full_config(rr, "video64k")
+
+
+@pytest.mark.slow
+def test_llama128k(rr):
+    check_full_config(rr, "llama128k")
