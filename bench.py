@@ -48,7 +48,8 @@ def workload_config(cfg: gen.Config, tau: float) -> dict:
             "structure": {0: "iid", 1: "planted sinks", 2: "planted sinks + local band", 3: "video frames"}[
                 cfg.structure],
             "L": cfg.L, "H": cfg.H, "Hkv": cfg.Hkv, "d": cfg.d, "B": cfg.B, "S": cfg.S, "tau": tau,
-            "l2": "inputs exceed L2 (q alone is %.2f GB > 126 MB)" % (cfg.L * cfg.H * cfg.d * 2 / 1e9),
+            "l2": ("inputs exceed L2: q alone is %.2f GB > 126 MB, no flush needed" % (cfg.L * cfg.H * cfg.d * 2 / 1e9)
+                   if cfg.L * cfg.H * cfg.d * 2 > 126e6 else "inputs fit in L2 (not flushed)"),
             "seed": cfg.seed}
 
 
@@ -152,7 +153,7 @@ def run_reference(args, cfg, tau, world):
     times = []
     res = None
     for it in range(args.warmup + args.steps):
-        res = oracle_sample(cfg, tau, q, k, v, heads=1, rows_per_head=args.ref_rows, seed=it)
+        res = oracle_sample(cfg, tau, q, k, v, heads=args.ref_heads, rows_per_head=args.ref_rows, seed=it)
         if it >= args.warmup:
             times.append(res["step_s"])
     step_s = statistics.mean(times)
@@ -347,7 +348,7 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res = oracle_sample(cfg, tau, q, k, v, heads=1, rows_per_head=args.ref_rows)
+        res = oracle_sample(cfg, tau, q, k, v, heads=args.ref_heads, rows_per_head=args.ref_rows)
         cpu = {k2: res[k2] for k2 in ("value", "unit", "cores", "kind", "sample")}
 
     if rank == 0:
@@ -375,7 +376,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="llama128k", choices=sorted(gen.CONFIGS))
     ap.add_argument("--tau", type=float, default=None)
-    ap.add_argument("--ref-rows", type=int, default=12)
+    ap.add_argument("--ref-heads", type=int, default=2, help="oracle sample: heads searched in full")
+    ap.add_argument("--ref-rows", type=int, default=16, help="oracle sample: attention rows per head")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

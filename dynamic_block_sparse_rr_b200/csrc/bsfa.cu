@@ -20,13 +20,17 @@
 // than 8 (a factor 256), which keeps P <= 256 and is exact after the final
 // division because P and l always use the same max.
 //
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer (one
-// thread; owns the 512-column TMEM allocation), warps 2-5 softmax group 0,
-// warps 6-9 softmax group 1.  TMEM columns: S_0 [0,128), S_1 [128,256),
-// O_0 [256,384), O_1 [384,512); P_x overwrites the first B/2 columns of S_x.
+// Warp roles (384 threads, three warpgroups): warp 0 TMA producer, warp 1 MMA
+// issuer (one thread; owns the 512-column TMEM allocation), warps 2-3 idle;
+// warps 4-7 softmax group 0, warps 8-11 softmax group 1.  The first warpgroup
+// gives registers back (setmaxnreg 72) so that the softmax groups can hold a
+// full 128-column score row (setmaxnreg 216): 128*72 + 256*216 = 384*168.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512);
+// P_x overwrites the first B/2 columns of S_x.
 // K/V tiles stream through a 4-stage shared-memory ring in the order the MMA
 // consumes them: K0, K1, V0, K2, V1, K3, ...
 #include <cuda_bf16.h>
+#include <stdlib.h>
 
 #include "rr_internal.h"
 #include "sm100.cuh"
@@ -35,8 +39,14 @@
 namespace rr {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kStages = 4;
+
+// 1: one exp2 pair in four runs on the FMA pipe (ex2_fma); 0 (default): all on
+// MUFU, which measured faster (the softmax is issue-bound, not MUFU-bound).
+#ifndef RR_MIX_EXP
+#define RR_MIX_EXP 0
+#endif
 
 template <int BN, int D>
 struct FaCfg {
@@ -59,17 +69,68 @@ struct FaCtrl {
   uint64_t p_full[2];
   uint64_t merge;
   uint64_t drain;
+  uint64_t never;      // fault injection: a barrier nothing arrives on
   uint32_t tmem_base;
   int abort;
   float2 ml[2][128];
 };
+
+// Exponentiate one row of scores into P (bf16, written to TMEM at p_col) and
+// return the row sum of P in fp32.
+template <int BN, bool kMixExp>
+__device__ __forceinline__ float softmax_store(const float (&s)[BN], float sl2, float m_run, uint32_t p_col) {
+  const uint64_t scale2 = f2pack(sl2, sl2);
+  const uint64_t negm2 = f2pack(-m_run, -m_run);
+  uint64_t acc[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) acc[j] = 0ull;   // (+0.0f, +0.0f)
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int jj = c * 16 + j;
+      float x0, x1;
+      f2unpack(fma2(f2pack(s[2 * jj], s[2 * jj + 1]), scale2, negm2), x0, x1);
+      float p0, p1;
+      if (kMixExp && (jj & 3) == 3) {
+        p0 = ex2_fma(x0);
+        p1 = ex2_fma(x1);
+      } else {
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
+      acc[j & 3] = add2(acc[j & 3], f2pack(p0, p1));
+      pk[j] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(p_col + c * 16, pk);
+  }
+  const uint64_t t = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+  float lo, hi;
+  f2unpack(t, lo, hi);
+  return lo + hi;
+}
+
+// Row max of BN scores: eight independent three-input max chains.
+template <int BN>
+__device__ __forceinline__ float row_max(const float (&s)[BN]) {
+  float m8[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m8[j] = fmaxf(s[2 * j], s[2 * j + 1]);
+#pragma unroll
+  for (int j = 16; j < BN; j += 16) {
+#pragma unroll
+    for (int a = 0; a < 8; ++a) m8[a] = max3(m8[a], s[j + 2 * a], s[j + 2 * a + 1]);
+  }
+  return max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+}
 
 template <int BN, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bsfa_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                 const __grid_constant__ CUtensorMap mv, const int32_t* __restrict__ count,
                 const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o, int H, int Hkv, int Nb,
-                float sl2, unsigned int* status, uint64_t limit_ns) {
+                float sl2, unsigned int* status, uint64_t limit_ns, int inject_stall) {
   using C = FaCfg<BN, D>;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, BN, false, false);
   constexpr uint32_t kIdO = idesc_bf16_f32(128, D, false, true);
@@ -103,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&ctl->merge), 256);
     mbar_init(smem_u32(&ctl->drain), 1);
+    mbar_init(smem_u32(&ctl->never), 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -115,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tm = ctl->tmem_base;
   const Guard guard{&ctl->abort, status, limit_ns};
-
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && cnt > 0) {
@@ -157,7 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && cnt > 0) {
       int k = 0;
-      bool ok = wait_bar(smem_u32(&ctl->q_full), 0, guard, 2);
+      bool ok = true;
+      // Injected fault (tests only): wait on a barrier that nothing arrives
+      // on; the bounded wait gives up, and the CTA takes its abort path.
+      if (inject_stall) ok = wait_bar(smem_u32(&ctl->never), 0, guard, 9);
+      if (ok) ok = wait_bar(smem_u32(&ctl->q_full), 0, guard, 2);
       tc_fence_after();
       auto issue_s = [&](int x) {
         const int st = k % kStages;
@@ -206,9 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_bar(smem_u32(&ctl->drain), 0, kDrainLimitNs);
     }
     __syncwarp();
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
     // ------------------------------------------------------------ softmax groups
-    const int x = (warp - 2) >> 2;              // group 0: warps 2-5, group 1: warps 6-9
+    const int x = (warp - 4) >> 2;              // group 0: warps 4-7, group 1: warps 8-11
     const int wq = warp & 3;                    // TMEM lane quarter
     const int row = wq * 32 + lane;             // row of the query tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -230,12 +299,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32x2(s_col, s_col + 32, raw);
       }
       float s[BN];
-      const bool diag = diag_last && t == cnt - 1;
 #pragma unroll
-      for (int j = 0; j < BN; ++j) s[j] = (diag && j > row) ? -INFINITY : __uint_as_float(raw[j]);
-      float mx = s[0];
+      for (int j = 0; j < BN; ++j) s[j] = __uint_as_float(raw[j]);
+      const bool diag = diag_last && t == cnt - 1;   // uniform across the CTA
+      if (diag) {
 #pragma unroll
-      for (int j = 1; j < BN; ++j) mx = fmaxf(mx, s[j]);
+        for (int j = 0; j < BN; ++j)
+          if (j > row) s[j] = -INFINITY;                // causal mask inside block J == I
+      }
+      const float mx = row_max<BN>(s);
       const float m_blk = mx * sl2;
       // lazy rescale: move the running max only when it grows by more than 2^8
       bool rescale = false;
@@ -251,18 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_run = m_blk;
         }
       }
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float p0 = ex2(fmaf(s[c * 32 + 2 * j], sl2, -m_run));
-          const float p1 = ex2(fmaf(s[c * 32 + 2 * j + 1], sl2, -m_run));
-          sum += p0 + p1;
-          pk[j] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(s_col + c * 16, pk);
+      // P = 2^(s*scale*log2e - m) on MUFU (optionally one pair in four on the FMA
+      // pipe outside the diagonal block, whose masked -inf entries stay on MUFU)
+      float sum;
+      if (diag) {
+        sum = softmax_store<BN, false>(s, sl2, m_run, s_col);
+      } else {
+        sum = softmax_store<BN, RR_MIX_EXP != 0>(s, sl2, m_run, s_col);
       }
       // O of this group is quiescent here (its last P V completed before this S
       // was signalled), and the next P V is issued only after p_full.
@@ -339,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BN, int D>
 cudaError_t launch_bsfa_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                           const int32_t* count, const int32_t* idx, void* o, int H, int Hkv, int Nb, float sl2,
-                          const DeviceGuardArgs& g, cudaStream_t stream) {
+                          const DeviceGuardArgs& g, int inject, cudaStream_t stream) {
   using C = FaCfg<BN, D>;
   static bool attr = false;
   if (!attr) {
@@ -349,7 +416,7 @@ cudaError_t launch_bsfa_t(const CUtensorMap& mq, const CUtensorMap& mk, const CU
     attr = true;
   }
   bsfa_kernel<BN, D><<<static_cast<unsigned>(H) * Nb, kThreads, C::kSmem, stream>>>(
-      mq, mk, mv, count, idx, static_cast<__nv_bfloat16*>(o), H, Hkv, Nb, sl2, g.status, g.limit_ns);
+      mq, mk, mv, count, idx, static_cast<__nv_bfloat16*>(o), H, Hkv, Nb, sl2, g.status, g.limit_ns, inject);
   return cudaGetLastError();
 }
 
@@ -364,10 +431,14 @@ cudaError_t launch_bsfa(const void* q, const void* k, const void* v, const int32
       !make_tmap_rows(&mv, v, L, Hkv, d, B))
     return cudaErrorInvalidValue;
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
-  if (B == 128 && d == 128) return launch_bsfa_t<128, 128>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, stream);
-  if (B == 128 && d == 64) return launch_bsfa_t<128, 64>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, stream);
-  if (B == 64 && d == 128) return launch_bsfa_t<64, 128>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, stream);
-  if (B == 64 && d == 64) return launch_bsfa_t<64, 64>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, stream);
+  // RR_DEBUG_STALL_WAIT=1 injects a wait that never completes (tests of the
+  // bounded-wait path); unset in normal use.
+  const char* inj = getenv("RR_DEBUG_STALL_WAIT");
+  const int inject = (inj && inj[0] == '1') ? 1 : 0;
+  if (B == 128 && d == 128) return launch_bsfa_t<128, 128>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, inject, stream);
+  if (B == 128 && d == 64) return launch_bsfa_t<128, 64>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, inject, stream);
+  if (B == 64 && d == 128) return launch_bsfa_t<64, 128>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, inject, stream);
+  if (B == 64 && d == 64) return launch_bsfa_t<64, 64>(mq, mk, mv, count, idx, o, H, Hkv, Nb, sl2, g, inject, stream);
   return cudaErrorInvalidValue;
 }
 
