@@ -18,11 +18,11 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librr.so")
 
-RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT = range(6)
+RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT, RR_ESCRATCH = range(7)
 
 # every symbol that include/rr.h declares
 EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status",
-           "rr_set_wait_limit_ns", "rr_status_string")
+           "rr_set_wait_limit_ns", "rr_status_string", "rr_search_static")
 
 
 class RRError(RuntimeError):
@@ -47,6 +47,8 @@ def lib() -> ctypes.CDLL:
         L.rr_sparse_attn.argtypes = [vp, vp, vp, i, i, i, i, i, vp, vp, vp, vp, sz, vp]
         L.rr_attention.argtypes = [vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp, vp, sz, vp]
         L.rr_check_status.argtypes = [vp, vp]
+        L.rr_search_static.argtypes = [vp, vp, i, i, i, i, i, i, f, vp, vp, vp]
+        L.rr_search_static.restype = ctypes.c_int
         L.rr_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.rr_set_wait_limit_ns.restype = ctypes.c_uint64
         L.rr_status_string.argtypes = [i]

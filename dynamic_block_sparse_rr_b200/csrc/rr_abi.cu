@@ -146,6 +146,7 @@ const char* rr_status_string(rr_status s) {
     case RR_EALIGN: return "misaligned pointer (16 bytes; workspace 256 bytes)";
     case RR_ECUDA: return "CUDA error";
     case RR_ETIMEOUT: return "device-side wait timed out";
+    case RR_ESCRATCH: return "shape needs more scratch than rr_search_static's 32 MiB array";
   }
   return "unknown status";
 }

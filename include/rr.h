@@ -46,7 +46,8 @@ typedef enum {
   RR_EUNSUPPORTED = 2,
   RR_EALIGN = 3,
   RR_ECUDA = 4,
-  RR_ETIMEOUT = 5
+  RR_ETIMEOUT = 5,
+  RR_ESCRATCH = 6   /* rr_search_static only: the shape needs more than its static scratch */
 } rr_status;
 
 /* Bytes of device workspace that rr_search / rr_sparse_attn / rr_attention
@@ -99,6 +100,29 @@ rr_status rr_check_status(void* workspace, void* stream);
 /* Sets the bound, in nanoseconds, of every device-side wait of later launches
  * (default 2e9).  Returns the previous bound.  Process-wide. */
 uint64_t rr_set_wait_limit_ns(uint64_t ns);
+
+/* The pattern search of rr_search, for callers that cannot allocate device
+ * memory or hand the library a workspace (for example an operator interface
+ * that passes only its input and output tensors, or a process whose device
+ * memory is entirely owned by another allocator).  The paper has no
+ * counterpart to this entry point; it only changes where the scratch lives.
+ *   Scratch: a file-scope device array of 32 MiB inside this library, which
+ *   every GPU that loads the library holds until the process exits.  Shapes
+ *   whose rr_workspace_size exceeds 32 MiB are rejected with RR_ESCRATCH before
+ *   anything is enqueued (e.g. H=32, Hkv=8, d=128, B=128, S=16 fits up to
+ *   L=32768; L=65536 and beyond do not).
+ *   Allocation: none (no cudaMalloc, cudaFree or allocating library call).  The
+ *   first call on each device resolves the array's device address with that
+ *   device current; make that first call before any stream capture.
+ *   Sharing: every call, on every stream, uses the same array and the array
+ *   keeps the last call's contents; calls that overlap on the GPU race, so
+ *   serialise them (one stream, or events).
+ *   Status: device-side timeouts land in the array's status word, which the
+ *   caller cannot name; use rr_search with a workspace when rr_check_status is
+ *   needed.
+ * Arguments, outputs and validation otherwise as rr_search (mass not offered). */
+rr_status rr_search_static(const void* q, const void* k, int L, int H, int Hkv, int d, int B, int S,
+                           float tau, int32_t* count, int32_t* idx, void* stream);
 
 /* Static string for a status code. */
 const char* rr_status_string(rr_status s);
