@@ -171,6 +171,22 @@ def run_reference(args, cfg, tau, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- ranks
+def aggregate(total_ms: float, e2e_ms: float, flops: float, world: int, device) -> tuple:
+    """Max over ranks of the timed regions, sum over ranks of the work.
+
+    Every rank calls this exactly once, after its own timing, so all ranks take
+    the same collective steps in the same order."""
+    import torch
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
+    w = torch.tensor([flops], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(t[1]), float(w[0])
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -283,19 +299,6 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
     flops = block_flops(cfg, visited)
     gpu_launches = 4 * args.steps   # pool, search, top-tau, attention per step
 
-    # max over ranks of the timed region; sum of the work
-    tot = torch.tensor([total_ms, flops], dtype=torch.float64, device=dev)
-    if world > 1:
-        mx = tot.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = tot.clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        total_ms_max, flops_all = float(mx[0]), float(sm[1])
-    else:
-        total_ms_max, flops_all = total_ms, flops
-    ms_per_step = total_ms_max / args.steps
-    value = flops_all / (ms_per_step / 1e3) / 1e12
-
     # dense baseline: the same attention kernel with every causal block on
     dense_ms = None
     if not args.no_dense:
@@ -331,10 +334,10 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = flops_all / (float(e2e_t[0]) / 1e3) / 1e12
+    total_ms_max, e2e_ms_max, flops_all = aggregate(total_ms, e2e_ms, flops, world, dev)
+    ms_per_step = total_ms_max / args.steps
+    value = flops_all / (ms_per_step / 1e3) / 1e12
+    e2e_value = flops_all / (e2e_ms_max / 1e3) / 1e12
     h2d = (qh.numel() + kh.numel() + vh.numel()) * 2
     d2h = oh.numel() * 2
     del qd2, kd2, vd2
@@ -359,9 +362,9 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
             "config": workload_config(cfg, tau),
             "search_ms": search_ms, "attn_ms": attn_ms, "search_share": search_ms / (search_ms + attn_ms),
             "dense_attn_ms": dense_ms, "dense_attn_tflops": dense_tflops if dense_ms else None,
-            "speedup_vs_dense": (dense_ms / ms_per_step) if dense_ms else None,
+            "speedup_vs_dense": (dense_ms / (total_ms / args.steps)) if dense_ms else None,
             "visited_blocks": visited, "visited_fraction": visited / (H * Nb * (Nb + 1) / 2),
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": float(e2e_t[0]),
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms_max,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": gpu_launches, "clocks": clk, "roofline": roofline, "cpu_baseline": cpu,
         }
