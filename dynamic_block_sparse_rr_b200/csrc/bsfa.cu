@@ -20,11 +20,13 @@
 // than 8 (a factor 256), which keeps P <= 256 and is exact after the final
 // division because P and l always use the same max.
 //
-// Warp roles (384 threads, three warpgroups): warp 0 TMA producer, warp 1 MMA
-// issuer (one thread; owns the 512-column TMEM allocation), warps 2-3 idle;
-// warps 4-7 softmax group 0, warps 8-11 softmax group 1.  The first warpgroup
-// gives registers back (setmaxnreg 72) so that the softmax groups can hold a
-// full 128-column score row (setmaxnreg 216): 128*72 + 256*216 = 384*168.
+// Warp roles (384 threads, three warpgroups): warp 0 TMA producer; warps 1 and
+// 3 MMA issuers (one thread each) for softmax groups 0 and 1, taking strict
+// turns by whole MMA brackets (warp 1 also owns the 512-column TMEM
+// allocation); warp 2 idle; warps 4-7 softmax group 0, warps 8-11 softmax
+// group 1.  The first warpgroup
+// gives registers back (setmaxnreg 48) so that the softmax groups can hold a
+// full 128-column score row (setmaxnreg 224): 128*48 + 256*224 <= 384*168.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512);
 // P_x overwrites the first B/2 columns of S_x.
 // K/V tiles stream through a 4-stage shared-memory ring in the order the MMA
@@ -42,10 +44,17 @@ namespace {
 constexpr int kThreads = 384;
 constexpr int kStages = 4;
 
-// 1: one exp2 pair in four runs on the FMA pipe (ex2_fma); 0 (default): all on
-// MUFU, which measured faster (the softmax is issue-bound, not MUFU-bound).
-#ifndef RR_MIX_EXP
-#define RR_MIX_EXP 0
+// Every RR_EMU_EVERY-th exp2 pair of a non-diagonal block runs on the FMA pipe
+// (ex2_fma_x2) instead of MUFU; 0 keeps every exp2 on MUFU.
+#ifndef RR_EMU_EVERY
+#define RR_EMU_EVERY 0
+#endif
+
+// 1: after a group's first block, exponentiate with the running max while the
+// block max is found alongside (rows whose max jumps are redone); 0 (default,
+// measured faster): max first.
+#ifndef RR_SPEC_MAX
+#define RR_SPEC_MAX 0
 #endif
 
 template <int BN, int D>
@@ -68,43 +77,57 @@ struct FaCtrl {
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t merge;
-  uint64_t drain;
+  uint64_t drain[2];
   uint64_t never;      // fault injection: a barrier nothing arrives on
   uint32_t tmem_base;
   int abort;
+  int turn;            // which issuer may issue its next MMA bracket (0 or 1)
+  int issuer_done[2];  // an issuer with no bracket left never takes the turn
   float2 ml[2][128];
 };
 
-// Exponentiate one row of scores into P (bf16, written to TMEM at p_col) and
-// return the row sum of P in fp32.
-template <int BN, bool kMixExp>
-__device__ __forceinline__ float softmax_store(const float (&s)[BN], float sl2, float m_run, uint32_t p_col) {
+// Exponentiate one row of scores into P = 2^(s*sl2 - m) (bf16, written to TMEM
+// at p_col) and return the row sum of P in fp32.  kEmu > 0 moves every kEmu-th
+// pair from MUFU to the FMA pipe (ex2_fma_x2); kMax also returns the row max of
+// s, computed on the ALU alongside the exponentials.
+template <int BN, int kEmu, bool kMax>
+__device__ __forceinline__ float exp_store(const float (&s)[BN], float sl2, float m_run, uint32_t p_col,
+                                           float& mx_out) {
   const uint64_t scale2 = f2pack(sl2, sl2);
   const uint64_t negm2 = f2pack(-m_run, -m_run);
   uint64_t acc[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) acc[j] = 0ull;   // (+0.0f, +0.0f)
+  float m8[8];
+  if constexpr (kMax) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m8[j] = -INFINITY;
+  }
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t pk[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int jj = c * 16 + j;
-      float x0, x1;
-      f2unpack(fma2(f2pack(s[2 * jj], s[2 * jj + 1]), scale2, negm2), x0, x1);
-      float p0, p1;
-      if (kMixExp && (jj & 3) == 3) {
-        p0 = ex2_fma(x0);
-        p1 = ex2_fma(x1);
+      if constexpr (kMax) m8[j & 7] = max3(m8[j & 7], s[2 * jj], s[2 * jj + 1]);
+      const uint64_t xp = fma2(f2pack(s[2 * jj], s[2 * jj + 1]), scale2, negm2);
+      uint64_t pp;
+      if (kEmu > 0 && (jj % (kEmu > 0 ? kEmu : 1)) == kEmu - 1) {
+        pp = ex2_fma_x2(xp);
       } else {
-        p0 = ex2(x0);
-        p1 = ex2(x1);
+        float x0, x1;
+        f2unpack(xp, x0, x1);
+        pp = f2pack(ex2(x0), ex2(x1));
       }
-      acc[j & 3] = add2(acc[j & 3], f2pack(p0, p1));
+      acc[j & 3] = add2(acc[j & 3], pp);
+      float p0, p1;
+      f2unpack(pp, p0, p1);
       pk[j] = pack_bf16x2(p0, p1);
     }
     tmem_st16(p_col + c * 16, pk);
   }
+  if constexpr (kMax)
+    mx_out = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
   const uint64_t t = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
   float lo, hi;
   f2unpack(t, lo, hi);
@@ -163,9 +186,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&ctl->p_full[x]), 128);
     }
     mbar_init(smem_u32(&ctl->merge), 256);
-    mbar_init(smem_u32(&ctl->drain), 1);
+    mbar_init(smem_u32(&ctl->drain[0]), 1);
+    mbar_init(smem_u32(&ctl->drain[1]), 1);
     mbar_init(smem_u32(&ctl->never), 1);
     ctl->abort = 0;
+    ctl->turn = 0;
+    ctl->issuer_done[0] = ctl->issuer_done[1] = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -178,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tm = ctl->tmem_base;
   const Guard guard{&ctl->abort, status, limit_ns};
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 48;\n" ::: "memory");
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && cnt > 0) {
@@ -205,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++k;
         return true;
       };
+      // tile order = MMA order: K0, K1, V0, K2, V1, K3, ...
       ok = load(&mk, sList[0]);
       if (ok && cnt > 1) ok = load(&mk, sList[1]);
       for (int t = 0; t < cnt && ok; ++t) {
@@ -216,66 +243,110 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_bar(smem_u32(&ctl->full[kk % kStages]), (kk / kStages) & 1, kDrainLimitNs);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && cnt > 0) {
-      int k = 0;
+  } else if (warp & 1) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 1 issues softmax group 0's MMAs, warp 3 group 1's.  A tcgen05.mma
+    // issue occupies its thread for nearly the MMA's own run time, so any other
+    // instruction between two MMAs of one thread (even a satisfied barrier
+    // test) leaves the tensor core idle.  The two issuers therefore take strict
+    // turns by whole brackets (P V of one block and S of that group's next):
+    // while one issues back to back, the other does its waits.  Strict turns
+    // also keep the two groups half a period apart.
+    const int x = warp >> 1;
+    const int n_x = x == 0 ? (cnt + 1) >> 1 : cnt >> 1;   // list positions x, x+2, ...
+    if (lane == 0 && n_x > 0) {
       bool ok = true;
       // Injected fault (tests only): wait on a barrier that nothing arrives
       // on; the bounded wait gives up, and the CTA takes its abort path.
       if (inject_stall) ok = wait_bar(smem_u32(&ctl->never), 0, guard, 9);
       if (ok) ok = wait_bar(smem_u32(&ctl->q_full), 0, guard, 2);
-      tc_fence_after();
-      auto issue_s = [&](int x) {
-        const int st = k % kStages;
-        if (!wait_bar(smem_u32(&ctl->full[st]), (k / kStages) & 1, guard, 3)) return false;
-        tc_fence_after();
-        const uint8_t* kt = sStage + st * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(smem_u32(sQ + (kk >> 2) * 128 * 128 + 32 * (kk & 3)), 16, 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(kt + (kk >> 2) * BN * 128 + 32 * (kk & 3)), 16, 1024);
-          umma_ss(tm + x * 128, ad, bd, kIdS, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(smem_u32(&ctl->empty[st]));
-        ++k;
-        return true;
+      // Descriptor bases, computed once.  K-major tiles step 32 bytes (2 in the
+      // start-address field) per 16-wide K slice and one 64-column atom per 4
+      // slices; the V tile (MN-major) steps 16 rows (128 in the field) per slice.
+      const uint32_t q_lo = sdesc_sw128_lo(smem_u32(sQ), 16);
+      const uint32_t k_lo = sdesc_sw128_lo(smem_u32(sStage), 16);
+      const uint32_t v_lo = sdesc_sw128_lo(smem_u32(sStage), BN * 128);
+      constexpr uint32_t q_hi = sdesc_sw128_hi(1024), k_hi = sdesc_sw128_hi(1024), v_hi = sdesc_sw128_hi(1024);
+      constexpr uint32_t kStageStep = C::kTileBytes >> 4;
+      const uint32_t s_tm = tm + x * 128, o_tm = tm + 256 + x * 128;
+      // Position of a tile in the producer's order: K0, K1 (if cnt > 1), then
+      // for t = 0..cnt-1: V(t), and K(t+2) while t+2 < cnt.
+      const int c1 = cnt > 1 ? 1 : 0, tail = cnt > 2 ? cnt - 2 : 0;
+      auto pos_v = [&](int t) { return 1 + c1 + t + (t < tail ? t : tail); };
+      auto pos_k = [&](int t) { return t < 2 ? t : pos_v(t - 2) + 1; };
+      auto wait_tile = [&](int pos, int site) {
+        return wait_bar(smem_u32(&ctl->full[pos % kStages]), (pos / kStages) & 1, guard, site);
       };
-      auto issue_pv = [&](int x, bool acc) {
-        const int st = k % kStages;
-        if (!wait_bar(smem_u32(&ctl->full[st]), (k / kStages) & 1, guard, 4)) return false;
-        tc_fence_after();
-        const uint8_t* vt = sStage + st * C::kTileBytes;
+      auto emit_s = [&](int t) {
+        const int st = pos_k(t) % kStages;
+        const uint32_t kb = k_lo + st * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(smem_u32(vt + kk * 16 * 128), BN * 128, 1024);
-          umma_ts(tm + 256 + x * 128, tm + x * 128 + kk * 8, bd, kIdO, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss_lh(s_tm, q_lo + (kk >> 2) * (128 * 128 >> 4) + 2 * (kk & 3), q_hi,
+                     kb + (kk >> 2) * (BN * 128 >> 4) + 2 * (kk & 3), k_hi, kIdS, kk > 0 ? 1u : 0u);
         umma_commit(smem_u32(&ctl->empty[st]));
-        ++k;
-        return true;
       };
-      if (ok) ok = issue_s(0);
-      if (ok) umma_commit(smem_u32(&ctl->s_full[0]));
-      if (ok && cnt > 1) {
-        ok = issue_s(1);
-        if (ok) umma_commit(smem_u32(&ctl->s_full[1]));
+      auto emit_pv = [&](int t, bool acc) {
+        const int st = pos_v(t) % kStages;
+        const uint32_t vb = v_lo + st * kStageStep;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts_lh(o_tm, s_tm + kk * 8, vb + kk * (16 * 128 >> 4), v_hi, kIdO, (acc || kk > 0) ? 1u : 0u);
+        umma_commit(smem_u32(&ctl->empty[st]));
+      };
+      volatile int* turn = &ctl->turn;
+      volatile int* other_done = &ctl->issuer_done[x ^ 1];
+      // Wait for this issuer's turn (bounded; the other issuer may have finished).
+      auto take_turn = [&]() {
+        const uint64_t t0 = global_ns();
+        for (uint32_t it = 0;; ++it) {
+          if (*turn == x || *other_done) return true;
+          if ((it & 255) == 255) {
+            if (*guard.abort) return false;
+            if (global_ns() - t0 > guard.limit_ns) {
+              *guard.abort = 1;
+              atomicCAS(guard.status, 0u, kStatusTimeout | (11u << 8));
+              return false;
+            }
+          }
+        }
+      };
+      auto give_turn = [&]() { *turn = x ^ 1; };
+      // first S of this group: issuer 0 goes first, then issuer 1
+      if (ok) ok = wait_tile(pos_k(x), 3);
+      if (ok) ok = take_turn();
+      if (ok) {
+        emit_s(x);
+        umma_commit(smem_u32(&ctl->s_full[x]));
+        give_turn();
       }
-      for (int t = 0; t < cnt && ok; ++t) {
-        const int x = t & 1, u = t >> 1;
-        if (!wait_bar(smem_u32(&ctl->p_full[x]), u & 1, guard, 5)) { ok = false; break; }
-        tc_fence_after();
-        ok = issue_pv(x, u > 0);
-        if (ok && t + 2 < cnt) ok = issue_s(x);
-        if (ok) umma_commit(smem_u32(&ctl->s_full[x]));
+      for (int i = 0; i < n_x && ok; ++i) {
+        const int t = 2 * i + x;
+        const bool more = i + 1 < n_x;
+        // everything this bracket needs, while the other issuer's bracket runs:
+        // the tiles first (they landed long ago; each satisfied test still
+        // costs the thread ~150 cycles), then P, then the turn
+        if (!wait_tile(pos_v(t), 4)) { ok = false; break; }
+        if (more && !wait_tile(pos_k(t + 2), 3)) { ok = false; break; }
+        if (!wait_bar(smem_u32(&ctl->p_full[x]), i & 1, guard, 5)) { ok = false; break; }
+        tc_fence_after();   // P was written to TMEM by the softmax threads
+        if (!take_turn()) { ok = false; break; }
+        emit_pv(t, i > 0);
+        if (more) emit_s(t + 2);
+        umma_commit(smem_u32(&ctl->s_full[x]));
+        if (!more) ctl->issuer_done[x] = 1;
+        give_turn();
       }
-      umma_commit(smem_u32(&ctl->drain));
-      drain_bar(smem_u32(&ctl->drain), 0, kDrainLimitNs);
+      if (!ok) ctl->issuer_done[x] = 1;
+      umma_commit(smem_u32(&ctl->drain[x]));
+      drain_bar(smem_u32(&ctl->drain[x]), 0, kDrainLimitNs);
+    } else if (lane == 0) {
+      ctl->issuer_done[x] = 1;   // no bracket for this group
     }
     __syncwarp();
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;\n" ::: "memory");
     // ------------------------------------------------------------ softmax groups
     const int x = (warp - 4) >> 2;              // group 0: warps 4-7, group 1: warps 8-11
     const int wq = warp & 3;                    // TMEM lane quarter
@@ -307,29 +378,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < BN; ++j)
           if (j > row) s[j] = -INFINITY;                // causal mask inside block J == I
       }
-      const float mx = row_max<BN>(s);
-      const float m_blk = mx * sl2;
-      // lazy rescale: move the running max only when it grows by more than 2^8
+      // Online softmax with a lazy rescale: the running max moves (and O is
+      // rescaled in TMEM) only when a row's block max exceeds it by more than 8.
+      // After the first block the exponentials start at once with the running
+      // max, the block max being found alongside them; the rare rows whose max
+      // jumps are then redone.  The first block and the masked diagonal block
+      // take the max first.
+      float sum, dummy;
       bool rescale = false;
       float alpha = 1.0f;
-      if (u == 0) {
-        m_run = m_blk;
+      if (u == 0 || diag || !RR_SPEC_MAX) {
+        const float m_blk = row_max<BN>(s) * sl2;
+        if (u == 0) {
+          m_run = m_blk;
+        } else {
+          const bool need = m_blk > m_run + kRescale;
+          rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = ex2(m_run - m_blk);
+            l_run *= alpha;
+            m_run = m_blk;
+          }
+        }
+        if (diag) {
+          sum = exp_store<BN, 0, false>(s, sl2, m_run, s_col, dummy);
+        } else {
+          sum = exp_store<BN, RR_EMU_EVERY, false>(s, sl2, m_run, s_col, dummy);
+        }
       } else {
+        float mx;
+        sum = exp_store<BN, RR_EMU_EVERY, true>(s, sl2, m_run, s_col, mx);
+        const float m_blk = mx * sl2;
         const bool need = m_blk > m_run + kRescale;
         rescale = __any_sync(0xffffffffu, need);
-        if (need) {
-          alpha = ex2(m_run - m_blk);
-          l_run *= alpha;
-          m_run = m_blk;
+        if (rescale) {
+          if (need) {
+            alpha = ex2(m_run - m_blk);
+            l_run *= alpha;
+            m_run = m_blk;
+          }
+          tmem_wait_st();
+          sum = exp_store<BN, RR_EMU_EVERY, false>(s, sl2, m_run, s_col, dummy);
         }
-      }
-      // P = 2^(s*scale*log2e - m) on MUFU (optionally one pair in four on the FMA
-      // pipe outside the diagonal block, whose masked -inf entries stay on MUFU)
-      float sum;
-      if (diag) {
-        sum = softmax_store<BN, false>(s, sl2, m_run, s_col);
-      } else {
-        sum = softmax_store<BN, RR_MIX_EXP != 0>(s, sl2, m_run, s_col);
       }
       // O of this group is quiescent here (its last P V completed before this S
       // was signalled), and the next P V is issued only after p_full.

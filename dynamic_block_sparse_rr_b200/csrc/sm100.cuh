@@ -51,6 +51,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `hint_ns` while
+// the phase is incomplete, so that a waiting warp does not spin and take issue
+// slots from the warps sharing its scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+#ifndef RR_WAIT_HINT_NS
+#define RR_WAIT_HINT_NS 20000
+#endif
+
 // Every wait in the kernels is bounded.  When one runs past `limit_ns` it
 // raises the CTA's shared abort flag and records the site in the global
 // status word; any other wait of the CTA that sees the flag also gives up, so
@@ -65,9 +84,13 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Gu
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
+    if (RR_WAIT_HINT_NS > 0) {
+      if (mbar_try_wait_sleep(bar, parity, RR_WAIT_HINT_NS)) return true;
+    } else {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      for (int i = 0; i < 32; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    }
     if (*g.abort) return false;
     if (global_ns() - t0 > g.limit_ns) {
       *g.abort = 1;
@@ -161,6 +184,31 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Same two MMAs with the 64-bit descriptors passed as (lo, hi) halves: callers
+// keep per-tile descriptor bases and step the start-address field (low word)
+// with 32-bit immediate adds, so little but the MMA itself sits in the issue
+// path.  The start-address field never carries into the high word.
+__device__ __forceinline__ void umma_ss_lh(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                           uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_lh(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread completes.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -187,6 +235,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
          (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// The two 32-bit halves of sdesc_sw128 (low: start address and LBO; high: SBO,
+// version 1 and the 128-byte swizzle layout type).
+__device__ __forceinline__ uint32_t sdesc_sw128_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sdesc_sw128_hi(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
 
 // TMEM address: lane in bits 16-31, column in bits 0-15.
@@ -323,6 +380,23 @@ __device__ __forceinline__ float ex2_fma(float x) {
   p = fmaf(p, f, 6.932609677e-01f);
   p = fmaf(p, f, 9.999280572e-01f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// ex2_fma on a packed pair (same arithmetic, f32x2 instructions).
+__device__ __forceinline__ uint64_t ex2_fma_x2(uint64_t xp) {
+  float x0, x1;
+  f2unpack(xp, x0, x1);
+  const uint64_t xc = f2pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t t = add2(xc, f2pack(12582912.0f, 12582912.0f));
+  const uint64_t f = fma2(add2(t, f2pack(-12582912.0f, -12582912.0f)), f2pack(-1.0f, -1.0f), xc);
+  uint64_t p = fma2(f2pack(5.517166853e-02f, 5.517166853e-02f), f, f2pack(2.426111251e-01f, 2.426111251e-01f));
+  p = fma2(p, f, f2pack(6.932609677e-01f, 6.932609677e-01f));
+  p = fma2(p, f, f2pack(9.999280572e-01f, 9.999280572e-01f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  return f2pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
 }
 
 // Two fp32 -> packed bf16x2 (lo in bits 0-15), round to nearest even.
