@@ -2,7 +2,8 @@
 // blocks (RRAttention abstract: "computing only half of the attention
 // blocks", "2.4x speedup at 128K"; Figure 2 stage 3; Figure 3a).
 //
-// One CTA per (head h, query block I): a 128-row query tile (the B = 64 case
+// One CTA per (head h, query block I), launched kv head by kv head, longest
+// rows first: a 128-row query tile (the B = 64 case
 // uses the first 64 rows), the key blocks J listed for (h, I) visited in
 // ascending order.  Both contractions per block run on tcgen05 with fp32
 // accumulators in TMEM:
@@ -167,9 +168,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   FaCtrl* ctl = reinterpret_cast<FaCtrl*>(smem + C::kCtrlOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int I = Nb - 1 - static_cast<int>(blockIdx.x / H);   // longer rows first
-  const int h = static_cast<int>(blockIdx.x % H);
-  const int kvh = h / (H / Hkv);
+  // CTA order: kv head by kv head, and inside one kv head longer rows first
+  // with the g query heads of a row side by side.  The CTAs resident at any time
+  // then share one kv head's K and V (64 MB at L = 128K, d = 128), which stay
+  // in L2 instead of being re-read from HBM by every row.
+  const int g = H / Hkv;
+  const int per_kv = g * Nb;
+  const int kvh = static_cast<int>(blockIdx.x / per_kv);
+  const int r = static_cast<int>(blockIdx.x % per_kv);
+  const int I = Nb - 1 - r / g;
+  const int h = kvh * g + r % g;
   const long long row_id = static_cast<long long>(h) * Nb + I;
   int cnt = count[row_id];
   cnt = cnt < 0 ? 0 : (cnt > Nb ? Nb : cnt);
