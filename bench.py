@@ -371,6 +371,33 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_recall(args, cfg, taus):
+    """Mask diagnostics: per tau, the RR mask's visited fraction and its recall of
+    the exact attention mass, next to the exact Top-tau selection (the search at
+    stride 1).  Prints one JSON line."""
+    import torch
+    import dynamic_block_sparse_rr_b200 as rr
+    q, k, _ = gen.make_config(cfg)
+    dev = torch.device("cuda", 0)
+    qd = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).to(dev)
+    kd = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).to(dev)
+    Nb = cfg.L // cfg.B
+    causal = cfg.H * Nb * (Nb + 1) / 2
+    m_exact = rr.exact_block_mass(qd, kd, cfg.B)
+    rows = []
+    for tau in taus:
+        c_rr, i_rr = rr.search(qd, kd, cfg.B, cfg.S, tau)
+        c_ex, i_ex = rr.search(qd, kd, cfg.B, 1, tau)
+        rec_rr = rr.mask_recall(m_exact, c_rr, i_rr)[:, :-1]
+        rec_ex = rr.mask_recall(m_exact, c_ex, i_ex)[:, :-1]
+        rows.append({"tau": tau, "visited_rr": c_rr.sum().item() / causal, "visited_exact": c_ex.sum().item() / causal,
+                     "recall_rr_mean": rec_rr.mean().item(), "recall_rr_min": rec_rr.min().item(),
+                     "recall_exact_mean": rec_ex.mean().item()})
+    torch.cuda.synchronize()
+    print(json.dumps({"diagnostic": "mask recall of exact attention mass (last query block excluded)",
+                      "config": workload_config(cfg, taus[0]), "rows": rows}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -383,6 +410,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=16, help="oracle sample: attention rows per head")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--recall", action="store_true",
+                    help="mask diagnostics instead of timing: recall of exact attention mass per tau")
     args = ap.parse_args()
     if args.warmup < 3:
         print("note: fewer than 3 warm-up steps requested", file=sys.stderr)
@@ -396,6 +425,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, cfg, tau, world)
+        return
+    if args.recall:
+        if rank == 0:
+            run_recall(args, cfg, list(cfg.taus) if args.tau is None else [tau])
         return
 
     if world > 1:

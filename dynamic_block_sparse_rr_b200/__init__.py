@@ -22,7 +22,7 @@ RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT, RR_ESCRATCH
 
 # every symbol that include/rr.h declares
 EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status",
-           "rr_set_wait_limit_ns", "rr_status_string", "rr_search_static")
+           "rr_set_wait_limit_ns", "rr_status_string", "rr_search_static", "rr_mask_recall")
 
 
 class RRError(RuntimeError):
@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
         L.rr_check_status.argtypes = [vp, vp]
         L.rr_search_static.argtypes = [vp, vp, i, i, i, i, i, i, f, vp, vp, vp]
         L.rr_search_static.restype = ctypes.c_int
+        L.rr_mask_recall.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.rr_mask_recall.restype = ctypes.c_int
         L.rr_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.rr_set_wait_limit_ns.restype = ctypes.c_uint64
         L.rr_status_string.argtypes = [i]
@@ -149,6 +151,28 @@ def attention(q, k, v, B: int, S: int, tau: float, out=None, count=None, idx=Non
                               count.data_ptr(), idx.data_ptr(), out.data_ptr(), ws.data_ptr(), ws.numel(),
                               _stream(stream)), "rr_attention")
     return out, count, idx
+
+
+def exact_block_mass(q, k, B: int, mass=None, stream=None):
+    """Exact full-attention block mass [H, Nb, Nb] fp32 (unnormalised, J <= I):
+    the search at stride S = 1, where every query is sampled and every key is its
+    own stride."""
+    L, H, Hkv, d = _shape(q, k)
+    Nb = L // B
+    if mass is None:
+        mass = torch.zeros((H, Nb, Nb), dtype=torch.float32, device=q.device)
+    search(q, k, B, 1, 1.0, mass=mass, stream=stream)
+    return mass
+
+
+def mask_recall(mass, count, idx, out=None, stream=None):
+    """Share of each row's mass kept by the mask -> recall [H, Nb] fp32."""
+    H, Nb = count.shape
+    if out is None:
+        out = torch.empty((H, Nb), dtype=torch.float32, device=count.device)
+    _check(lib().rr_mask_recall(mass.data_ptr(), count.data_ptr(), idx.data_ptr(), H, Nb, out.data_ptr(),
+                                _stream(stream)), "rr_mask_recall")
+    return out
 
 
 def check_status(ws, stream=None) -> int:

@@ -122,6 +122,16 @@ rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H
   return RR_OK;
 }
 
+rr_status rr_mask_recall(const float* mass, const int32_t* count, const int32_t* idx, int H, int Nb,
+                         float* recall, void* stream) {
+  if (!mass || !count || !idx || !recall || H <= 0 || Nb <= 0) return RR_EINVAL;
+  if (Nb > rr::kMaxBlocks) return RR_EUNSUPPORTED;
+  if (!aligned16(mass) || !aligned16(count) || !aligned16(idx) || !aligned16(recall)) return RR_EALIGN;
+  if (rr::launch_mask_recall(mass, count, idx, H, Nb, recall, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RR_ECUDA;
+  return RR_OK;
+}
+
 rr_status rr_check_status(void* workspace, void* stream) {
   if (!workspace) return RR_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

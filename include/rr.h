@@ -92,6 +92,17 @@ rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H
                        int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/* Mask diagnostics (the synthetic counterpart of the pattern visualisations,
+ * Figures 4 and 5: full-attention ground truth against the RR selection).
+ * recall[h*Nb+I] = sum of mass[h,I,J] over the J listed in (count, idx) for row
+ * (h, I), divided by the sum of mass[h,I,J] over J <= I.  `mass` is an
+ * unnormalised block mass [H, Nb, Nb] fp32 (entries J <= I read), e.g. the
+ * `mass` output of rr_search at S = 1, which is the exact full-attention block
+ * mass.  All pointers are device memory; recall is [H, Nb] fp32, caller-owned.
+ * List entries outside [0, I] are ignored.  Asynchronous on `stream`. */
+rr_status rr_mask_recall(const float* mass, const int32_t* count, const int32_t* idx, int H, int Nb,
+                         float* recall, void* stream);
+
 /* Synchronises `stream`, returns the device-side status recorded since the
  * last rr_* call that started on this workspace (RR_OK or RR_ETIMEOUT), and
  * RR_ECUDA if the stream reports an error. */

@@ -201,6 +201,26 @@ def sparse_attention(Q, K, V, count, idx, B: int, rows=None) -> np.ndarray:
     return O
 
 
+# ------------------------------------------------ mask diagnostics (recall)
+def exact_block_mass(Q, K, B: int) -> np.ndarray:
+    """Exact full-attention block mass: the R3-R5 definitions at S = 1, where every
+    query is sampled and every key is its own stride (pinned against the attention
+    matrix of torch's scaled_dot_product_attention)."""
+    return block_mass(Q, K, B, 1)
+
+
+def mask_recall(M: np.ndarray, count: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """recall[h, I] = sum of M[h, I, J] over the selected J / sum over J <= I."""
+    H, Nb, _ = M.shape
+    m = normalise_mass(M)
+    out = np.zeros((H, Nb), dtype=np.float64)
+    for h in range(H):
+        for I in range(Nb):
+            sel = idx[h, I, :count[h, I]]
+            out[h, I] = m[h, I, sel].sum()
+    return out
+
+
 # -------------------------------------------------------- R9 comparison band
 def band_blocks(m_row: np.ndarray, I: int, tau: float, band: float = 1e-4, tie: float = 1e-6):
     """Blocks of row I whose selection may legitimately differ (R9).

@@ -289,3 +289,31 @@ def test_band_blocks_flags_the_cut():
     assert 1 in near                                     # running sum 0.94995 sits at tau
     near, ties = oracle.band_blocks(np.array([0.6, 0.2, 0.2]), 2, 0.7)
     assert ties == {1, 2}
+
+
+# ------------------------------------------------------------ mask diagnostics
+def test_recall_of_full_mask_is_one_and_top_tau_reaches_tau():
+    L, H, Hkv, d, B = 256, 2, 1, 16, 32
+    Q, K = _rand((L, H, d), 50), _rand((L, Hkv, d), 51) * 2.0
+    M = oracle.exact_block_mass(Q, K, B)
+    Nb = L // B
+    c_full, i_full = oracle.full_causal_mask(H, Nb)
+    assert np.allclose(oracle.mask_recall(M, c_full, i_full), 1.0, atol=1e-12)
+    for tau in (0.3, 0.8, 0.95):
+        c, i = oracle.select(oracle.normalise_mass(M), tau)
+        rec = oracle.mask_recall(M, c, i)
+        assert np.all(rec[:, :-1] >= tau - 1e-12)          # Top-tau of the exact mass reaches tau
+        assert np.allclose(rec[:, -1], 1.0)                  # protected last row
+
+
+def test_recall_of_single_block_equals_its_exact_share():
+    L, H, d, B = 128, 1, 8, 32
+    Q, K = _rand((L, H, d), 52), _rand((L, H, d), 53)
+    A = _sdpa_probs(Q, K)[0]                                # exact attention probabilities
+    M = oracle.exact_block_mass(Q, K, B)
+    count = np.ones((1, 4), np.int32)
+    idx = np.zeros((1, 4, 4), np.int32)                      # keep only J = 0 in every row
+    rec = oracle.mask_recall(M, count, idx)
+    for I in range(4):
+        want = A[I * B:(I + 1) * B, 0:B].sum() / B
+        assert abs(rec[0, I] - want) < 1e-12

@@ -237,3 +237,50 @@ def test_video64k(rr):
 @pytest.mark.slow
 def test_llama128k(rr):
     check_full_config(rr, "llama128k")
+
+
+# ------------------------------------------------------------ edge cases
+def test_small_tau_single_block_rows(rr):
+    """tau near 0: every row but the protected last one keeps exactly its heaviest block."""
+    rep = check_case(rr, 2048, 4, 2, 128, 128, 16, 1e-4, gen.PLANTED, seed=8)
+    assert rep[1e-4]["blocks_fail"] == 0
+
+
+@pytest.mark.slow
+def test_maximum_block_count(rr):
+    """Nb = 4096, the largest the ABI accepts (L = 262144 with B = 64): the Top-tau sort runs on
+    4096-entry rows and the attention kernel holds a 4096-entry block list."""
+    L, H, Hkv, d, B, S, tau = 262144, 1, 1, 64, 64, 4, 0.9
+    q, k, v = gen.make_qkv(L, H, Hkv, d, gen.PLANTED_BAND, 12)
+    Q, K, V = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k), gen.bf16_bits_to_f32(v)
+    count, idx, M_g, o = run_gpu(rr, to_dev(q), to_dev(k), to_dev(v), B, S, tau)
+    Nb = L // B
+    assert Nb == 4096
+    check_mask_format(count, idx)
+    m_o = oracle.normalise_mass(oracle.block_mass(Q, K, B, S))
+    count_o, idx_o = oracle.select(m_o, tau)
+    st = compare_masks(count, idx, count_o, idx_o, m_o, tau)
+    assert st["blocks_fail"] == 0, st
+    rows = [(0, 0), (0, Nb - 1), (0, Nb - 2), (0, 2048), (0, 17)]
+    O_ref = oracle.sparse_attention(Q, K, V, count, idx, B, rows=rows)
+    mx, mean = output_errors(gpu_o_f32(o), O_ref)
+    assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
+    print("Nb=4096", st, mx, mean)
+
+
+# ------------------------------------------------------------ mask diagnostics
+@pytest.mark.parametrize("L,H,Hkv,d,B,S,tau", [(2048, 4, 2, 128, 128, 16, 0.9), (1024, 4, 4, 64, 64, 4, 0.9)])
+def test_mask_recall_matches_oracle(rr, L, H, Hkv, d, B, S, tau):
+    q, k, _ = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 13)
+    Q, K = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k)
+    qd, kd = to_dev(q), to_dev(k)
+    count, idx = rr.search(qd, kd, B, S, tau)
+    M_g = rr.exact_block_mass(qd, kd, B)
+    rec = rr.mask_recall(M_g, count, idx).cpu().numpy()
+    M_o = oracle.exact_block_mass(Q, K, B)
+    tri = np.tri(L // B, dtype=bool)[None]
+    assert np.max(np.abs(np.where(tri, oracle.normalise_mass(M_g.cpu().numpy().astype(np.float64))
+                                  - oracle.normalise_mass(M_o), 0.0))) <= MASS_ERR
+    rec_o = oracle.mask_recall(M_o, count.cpu().numpy(), idx.cpu().numpy())
+    assert np.max(np.abs(rec - rec_o)) <= 1e-5
+    assert np.all(rec[:, -1] > 1 - 1e-6)
