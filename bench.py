@@ -371,7 +371,7 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
-def run_recall(args, cfg, taus):
+def run_recall(args, cfg, taus, variants=(0,)):
     """Mask diagnostics: per tau, the RR mask's visited fraction and its recall of
     the exact attention mass, next to the exact Top-tau selection (the search at
     stride 1).  Prints one JSON line."""
@@ -386,16 +386,40 @@ def run_recall(args, cfg, taus):
     m_exact = rr.exact_block_mass(qd, kd, cfg.B)
     rows = []
     for tau in taus:
-        c_rr, i_rr = rr.search(qd, kd, cfg.B, cfg.S, tau)
         c_ex, i_ex = rr.search(qd, kd, cfg.B, 1, tau)
-        rec_rr = rr.mask_recall(m_exact, c_rr, i_rr)[:, :-1]
         rec_ex = rr.mask_recall(m_exact, c_ex, i_ex)[:, :-1]
-        rows.append({"tau": tau, "visited_rr": c_rr.sum().item() / causal, "visited_exact": c_ex.sum().item() / causal,
-                     "recall_rr_mean": rec_rr.mean().item(), "recall_rr_min": rec_rr.min().item(),
-                     "recall_exact_mean": rec_ex.mean().item()})
+        row = {"tau": tau, "visited_exact": c_ex.sum().item() / causal, "recall_exact_mean": rec_ex.mean().item()}
+        for flags in variants:
+            c_rr, i_rr = rr.search_variant(qd, kd, cfg.B, cfg.S, tau, flags)
+            rec_rr = rr.mask_recall(m_exact, c_rr, i_rr)[:, :-1]
+            tag = variant_name(flags)
+            row.update({f"visited_{tag}": c_rr.sum().item() / causal, f"recall_{tag}_mean": rec_rr.mean().item(),
+                         f"recall_{tag}_min": rec_rr.min().item()})
+        rows.append(row)
+    # search time per variant (device events; one warm call first)
+    search_ms = {}
+    for flags in variants:
+        ws = rr.workspace(cfg.L, cfg.H, cfg.Hkv, cfg.d, cfg.B, cfg.S, dev, flags=flags)
+        count, idx = rr.empty_mask(cfg.H, Nb, dev)
+        rr.search_variant(qd, kd, cfg.B, cfg.S, taus[0], flags, count, idx, ws=ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(5):
+            rr.search_variant(qd, kd, cfg.B, cfg.S, taus[0], flags, count, idx, ws=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        search_ms[variant_name(flags)] = e0.elapsed_time(e1) / 5
+        if rr.check_status(ws) != rr.RR_OK:
+            raise RuntimeError("device-side wait timed out")
     torch.cuda.synchronize()
     print(json.dumps({"diagnostic": "mask recall of exact attention mass (last query block excluded)",
-                      "config": workload_config(cfg, taus[0]), "rows": rows}), flush=True)
+                      "config": workload_config(cfg, taus[0]), "rows": rows, "search_ms": search_ms}), flush=True)
+
+
+def variant_name(flags: int) -> str:
+    """rr: the plain search; rot / sk / gqa: the sampling variants of rr_search_variant."""
+    parts = [n for bit, n in ((1, "rot"), (2, "sk"), (4, "gqa")) if flags & bit]
+    return "+".join(parts) if parts else "rr"
 
 
 def main():
@@ -412,6 +436,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--recall", action="store_true",
                     help="mask diagnostics instead of timing: recall of exact attention mass per tau")
+    ap.add_argument("--variants", default="0",
+                    help="with --recall: comma-separated sampling-variant flags (1 rotate, 2 sampled keys, "
+                         "4 GQA mask; 0 the plain search)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("note: fewer than 3 warm-up steps requested", file=sys.stderr)
@@ -428,7 +455,8 @@ def main():
         return
     if args.recall:
         if rank == 0:
-            run_recall(args, cfg, list(cfg.taus) if args.tau is None else [tau])
+            run_recall(args, cfg, list(cfg.taus) if args.tau is None else [tau],
+                       [int(x) for x in args.variants.split(",")])
         return
 
     if world > 1:

@@ -22,7 +22,11 @@ RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT, RR_ESCRATCH
 
 # every symbol that include/rr.h declares
 EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status",
-           "rr_set_wait_limit_ns", "rr_status_string", "rr_search_static", "rr_mask_recall")
+           "rr_set_wait_limit_ns", "rr_status_string", "rr_search_static", "rr_mask_recall",
+           "rr_workspace_size_variant", "rr_search_variant")
+
+# sampling-variant flags of rr_search_variant (rr.h)
+VAR_ROTATE, VAR_SAMPLED_KEYS, VAR_GQA_MASK = 1, 2, 4
 
 
 class RRError(RuntimeError):
@@ -51,6 +55,11 @@ def lib() -> ctypes.CDLL:
         L.rr_search_static.restype = ctypes.c_int
         L.rr_mask_recall.argtypes = [vp, vp, vp, i, i, vp, vp]
         L.rr_mask_recall.restype = ctypes.c_int
+        u = ctypes.c_uint
+        L.rr_workspace_size_variant.argtypes = [i, i, i, i, i, i, u, ctypes.POINTER(sz)]
+        L.rr_workspace_size_variant.restype = ctypes.c_int
+        L.rr_search_variant.argtypes = [vp, vp, i, i, i, i, i, i, f, u, vp, vp, vp, vp, sz, vp]
+        L.rr_search_variant.restype = ctypes.c_int
         L.rr_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.rr_set_wait_limit_ns.restype = ctypes.c_uint64
         L.rr_status_string.argtypes = [i]
@@ -97,9 +106,18 @@ def workspace_size(L: int, H: int, Hkv: int, d: int, B: int, S: int) -> int:
     return n.value
 
 
-def workspace(L: int, H: int, Hkv: int, d: int, B: int, S: int, device=None) -> torch.Tensor:
-    """A device workspace (uint8) of the size the operator needs."""
-    return torch.empty(workspace_size(L, H, Hkv, d, B, S), dtype=torch.uint8, device=device or "cuda")
+def workspace(L: int, H: int, Hkv: int, d: int, B: int, S: int, device=None, flags: int = 0) -> torch.Tensor:
+    """A device workspace (uint8) of the size the operator needs (for the sampling
+    variant ``flags`` when given)."""
+    n = workspace_size(L, H, Hkv, d, B, S) if flags == 0 else workspace_size_variant(L, H, Hkv, d, B, S, flags)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def workspace_size_variant(L: int, H: int, Hkv: int, d: int, B: int, S: int, flags: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().rr_workspace_size_variant(L, H, Hkv, d, B, S, int(flags), ctypes.byref(n)),
+           "rr_workspace_size_variant")
+    return n.value
 
 
 def empty_mask(H: int, Nb: int, device=None):
@@ -119,6 +137,23 @@ def search(q, k, B: int, S: int, tau: float, count=None, idx=None, mass=None, ws
         ws = workspace(L, H, Hkv, d, B, S, q.device)
     _check(lib().rr_search(q.data_ptr(), k.data_ptr(), L, H, Hkv, d, B, S, float(tau), count.data_ptr(),
                            idx.data_ptr(), _ptr(mass), ws.data_ptr(), ws.numel(), _stream(stream)), "rr_search")
+    return count, idx
+
+
+def search_variant(q, k, B: int, S: int, tau: float, flags: int, count=None, idx=None, mass=None, ws=None,
+                   stream=None):
+    """Pattern search with the sampling variants ``flags`` (VAR_ROTATE,
+    VAR_SAMPLED_KEYS, VAR_GQA_MASK, or-ed) -> (count, idx).  ``mass`` receives the
+    per-head block masses."""
+    L, H, Hkv, d = _shape(q, k)
+    Nb = L // B
+    if count is None or idx is None:
+        count, idx = empty_mask(H, Nb, q.device)
+    if ws is None:
+        ws = workspace(L, H, Hkv, d, B, S, q.device, flags=flags)
+    _check(lib().rr_search_variant(q.data_ptr(), k.data_ptr(), L, H, Hkv, d, B, S, float(tau), int(flags),
+                                   count.data_ptr(), idx.data_ptr(), _ptr(mass), ws.data_ptr(), ws.numel(),
+                                   _stream(stream)), "rr_search_variant")
     return count, idx
 
 

@@ -15,19 +15,30 @@ constexpr size_t kAlign = 256;
 
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+constexpr unsigned kVarAll = RR_VAR_ROTATE | RR_VAR_SAMPLED_KEYS | RR_VAR_GQA_MASK;
+
+// Workspace regions (byte offsets).  With flags 0 only status, khi, klo and mass
+// are present, in that order (the rr_search layout).
 struct Layout {
-  size_t status, khi, klo, mass, total;
+  size_t status, khi, klo, qs, ks, mass, gmass, total;
 };
 
-Layout carve(int L, int H, int Hkv, int d, int B, int S) {
+Layout carve(int L, int H, int Hkv, int d, int B, int S, unsigned flags = 0) {
   Layout w;
   const size_t Ns = static_cast<size_t>(L / S), Nb = static_cast<size_t>(L / B);
-  const size_t kbar = round_up(Ns * Hkv * d * 2);
+  const bool pooled = !(flags & RR_VAR_SAMPLED_KEYS);
+  const bool rotate = (flags & RR_VAR_ROTATE) != 0;
+  const size_t kbar = pooled ? round_up(Ns * Hkv * d * 2) : 0;
+  const size_t gathered = round_up(Ns * H * d * 2);
+  size_t off = kAlign;
   w.status = 0;
-  w.khi = kAlign;
-  w.klo = w.khi + kbar;
-  w.mass = w.klo + kbar;
-  w.total = w.mass + round_up(static_cast<size_t>(H) * Nb * Nb * 4);
+  w.khi = off; off += kbar;
+  w.klo = off; off += kbar;
+  w.qs = off; off += rotate ? gathered : 0;
+  w.ks = off; off += (rotate && !pooled) ? gathered : 0;
+  w.mass = off; off += round_up(static_cast<size_t>(H) * Nb * Nb * 4);
+  w.gmass = off; off += (flags & RR_VAR_GQA_MASK) ? round_up(static_cast<size_t>(Hkv) * Nb * Nb * 4) : 0;
+  w.total = off;
   return w;
 }
 
@@ -64,27 +75,67 @@ rr_status rr_workspace_size(int L, int H, int Hkv, int d, int B, int S, size_t* 
   return RR_OK;
 }
 
-rr_status rr_search(const void* q, const void* k, int L, int H, int Hkv, int d, int B, int S, float tau,
-                    int32_t* count, int32_t* idx, float* mass, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+rr_status rr_workspace_size_variant(int L, int H, int Hkv, int d, int B, int S, unsigned flags, size_t* bytes) {
+  if (!bytes || (flags & ~kVarAll)) return RR_EINVAL;
+  rr_status st = check_shape(L, H, Hkv, d, B, S, true);
+  if (st != RR_OK) return st;
+  *bytes = carve(L, H, Hkv, d, B, S, flags).total;
+  return RR_OK;
+}
+
+rr_status rr_search_variant(const void* q, const void* k, int L, int H, int Hkv, int d, int B, int S, float tau,
+                            unsigned flags, int32_t* count, int32_t* idx, float* mass, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (flags & ~kVarAll) return RR_EINVAL;
   rr_status st = check_shape(L, H, Hkv, d, B, S, true);
   if (st != RR_OK) return st;
   if (!(tau > 0.0f) || tau != tau) return RR_EINVAL;
   if (!q || !k || !count || !idx) return RR_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(count) || !aligned16(idx) || (mass && !aligned16(mass)))
     return RR_EALIGN;
-  const Layout w = carve(L, H, Hkv, d, B, S);
+  const Layout w = carve(L, H, Hkv, d, B, S, flags);
   if ((st = check_ws(workspace, workspace_bytes, w)) != RR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   unsigned int* status = reinterpret_cast<unsigned int*>(ws + w.status);
   float* m = mass ? mass : reinterpret_cast<float*>(ws + w.mass);
   const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
+  const bool rotate = (flags & RR_VAR_ROTATE) != 0, sampled = (flags & RR_VAR_SAMPLED_KEYS) != 0;
+  const int g_heads = H / Hkv;
   if (cudaMemsetAsync(status, 0, sizeof(unsigned int), s) != cudaSuccess) return RR_ECUDA;
-  if (rr::launch_pool_keys(k, ws + w.khi, ws + w.klo, L, Hkv, d, S, s) != cudaSuccess) return RR_ECUDA;
-  if (rr::launch_search(q, ws + w.khi, ws + w.klo, m, L, H, Hkv, d, B, S, g, s) != cudaSuccess) return RR_ECUDA;
-  if (rr::launch_top_tau(m, H, L / B, tau, count, idx, s) != cudaSuccess) return RR_ECUDA;
+  rr::SearchSources src{q, ws + w.khi, ws + w.klo, 0, 0};
+  if (rotate) {
+    if (rr::launch_gather_rotated(q, ws + w.qs, L, H, H, 1, d, S, s) != cudaSuccess) return RR_ECUDA;
+    src.q = ws + w.qs;
+    src.q_mode = 1;
+  }
+  if (!sampled) {
+    if (rr::launch_pool_keys(k, ws + w.khi, ws + w.klo, L, Hkv, d, S, s) != cudaSuccess) return RR_ECUDA;
+  } else if (rotate) {
+    if (rr::launch_gather_rotated(k, ws + w.ks, L, H, Hkv, g_heads, d, S, s) != cudaSuccess) return RR_ECUDA;
+    src.k_a = src.k_b = ws + w.ks;
+    src.k_mode = 2;
+  } else {
+    src.k_a = src.k_b = k;
+    src.k_mode = 1;
+  }
+  if (rr::launch_search(src, m, L, H, Hkv, d, B, S, g, s) != cudaSuccess) return RR_ECUDA;
+  const int Nb = L / B;
+  if (flags & RR_VAR_GQA_MASK) {
+    float* gm = reinterpret_cast<float*>(ws + w.gmass);
+    if (rr::launch_group_mass(m, gm, Hkv, g_heads, Nb, s) != cudaSuccess) return RR_ECUDA;
+    if (rr::launch_top_tau(gm, Hkv, Nb, tau, count, idx, g_heads, s) != cudaSuccess) return RR_ECUDA;
+  } else {
+    if (rr::launch_top_tau(m, H, Nb, tau, count, idx, 1, s) != cudaSuccess) return RR_ECUDA;
+  }
   return RR_OK;
+}
+
+rr_status rr_search(const void* q, const void* k, int L, int H, int Hkv, int d, int B, int S, float tau,
+                    int32_t* count, int32_t* idx, float* mass, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  return rr_search_variant(q, k, L, H, Hkv, d, B, S, tau, 0u, count, idx, mass, workspace, workspace_bytes,
+                           stream);
 }
 
 rr_status rr_sparse_attn(const void* q, const void* k, const void* v, int L, int H, int Hkv, int d, int B,

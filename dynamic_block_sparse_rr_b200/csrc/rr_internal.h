@@ -18,11 +18,33 @@ cudaError_t launch_pool_keys(const void* k, void* khi, void* klo, int L, int Hkv
                              cudaStream_t stream);
 
 // Sampled-score search: block mass[h, I, J] (unnormalised) for J <= I.
-cudaError_t launch_search(const void* q, const void* khi, const void* klo, float* mass, int L, int H,
-                          int Hkv, int d, int B, int S, const DeviceGuardArgs& g, cudaStream_t stream);
+//   q_mode 0: q is [L, H, d], rows read at offset h mod S in each stride;
+//          1: q holds the sampled rows, gathered into [Ns, H, d].
+//   k_mode 0: k_a / k_b are the stride means' bf16 (hi, lo) parts [Ns, Hkv, d];
+//          1: k_a is k [L, Hkv, d], one key per stride at offset h mod S;
+//          2: k_a holds the sampled keys, gathered into [Ns, H, d].
+struct SearchSources {
+  const void* q;
+  const void* k_a;
+  const void* k_b;
+  int q_mode;
+  int k_mode;
+};
+cudaError_t launch_search(const SearchSources& src, float* mass, int L, int H, int Hkv, int d, int B, int S,
+                          const DeviceGuardArgs& g, cudaStream_t stream);
+
+// Rows at the rotating offsets: dst[i, h, :] = src[i*S + (h + i) mod S, h / div, :]
+// for i < L/S, h < H (src [L, heads, d], dst [L/S, H, d], bf16).
+cudaError_t launch_gather_rotated(const void* src, void* dst, int L, int H, int src_heads, int div, int d, int S,
+                                  cudaStream_t stream);
+
+// GQA group mass: dst[kv, I, J] = sum of src[kv*g + t, I, J] over t < g (all I, J).
+cudaError_t launch_group_mass(const float* src, float* dst, int Hkv, int g, int Nb, cudaStream_t stream);
 
 // Adaptive Top-tau with protection of the last query block.
-cudaError_t launch_top_tau(const float* mass, int H, int Nb, float tau, int32_t* count, int32_t* idx,
+// rows = heads of `mass` ([rows, Nb, Nb]); each row's selection is written to the
+// rep output heads rows*rep.. (rep = 1: one output head per mass head).
+cudaError_t launch_top_tau(const float* mass, int rows, int Nb, float tau, int32_t* count, int32_t* idx, int rep,
                            cudaStream_t stream);
 
 // Causal block-sparse attention over the mask.

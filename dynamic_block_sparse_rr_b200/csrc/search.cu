@@ -61,7 +61,7 @@ template <int D, int LOGR>
 __global__ void __launch_bounds__(kThreads, 2)
     search_kernel(const __grid_constant__ CUtensorMap mqs, const __grid_constant__ CUtensorMap mkh,
                   const __grid_constant__ CUtensorMap mkl, float* __restrict__ mass, int H, int Hkv, int S,
-                  int Ns, int Nb, float sl2, unsigned int* status, uint64_t limit_ns) {
+                  int Ns, int Nb, float sl2, int q_mode, int k_mode, unsigned int* status, uint64_t limit_ns) {
   using C = SearchCfg<D>;
   constexpr int R = 1 << LOGR;                 // sampled rows (and strides) per block
   constexpr int GPT = kTile / R;               // key blocks per 128-stride tile
@@ -81,6 +81,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int kvh = h / (H / Hkv);
   const int n_key_tiles = rt + 1;
   const int n_seq = 2 * n_key_tiles;           // pass 1 then pass 2
+  // q_mode 0: sampled rows read through the 4D view (d, H, S, Ns) at offset h mod S;
+  //        1: rows gathered beforehand into [Ns, H, d] (rotating offsets).
+  // k_mode 0: stride means as a bf16 (hi, lo) pair [Ns, Hkv, d], two MMA chains;
+  //        1: one sampled key per stride through the 4D view of k at offset h mod S;
+  //        2: sampled keys gathered beforehand into [Ns, H, d].
+  const int parts = k_mode == 0 ? 2 : 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -115,21 +121,32 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_prefetch_desc(&mkl);
       const uint32_t qb = smem_u32(&ctl->q_full);
       mbar_expect_tx(qb, C::kTileBytes);
-      for (int a = 0; a < D / 64; ++a)
-        tma_load_4d(smem_u32(sQ + a * kTile * 128), &mqs, qb, a * 64, h, h % S, rt * kTile);
+      for (int a = 0; a < D / 64; ++a) {
+        if (q_mode == 0)
+          tma_load_4d(smem_u32(sQ + a * kTile * 128), &mqs, qb, a * 64, h, h % S, rt * kTile);
+        else
+          tma_load_3d(smem_u32(sQ + a * kTile * 128), &mqs, qb, a * 64, h, rt * kTile);
+      }
       int k = 0;
       bool ok = true;
       for (int n = 0; n < n_seq && ok; ++n) {
         const int c = n % n_key_tiles;
-        for (int part = 0; part < 2 && ok; ++part) {
+        for (int part = 0; part < parts && ok; ++part) {
           const int st = k % C::kStages;
           const uint32_t ph = (k / C::kStages) & 1;
           if (!wait_bar(smem_u32(&ctl->empty[st]), ph ^ 1, guard, 1)) { ok = false; break; }
           const uint32_t fb = smem_u32(&ctl->full[st]);
           mbar_expect_tx(fb, C::kTileBytes);
           uint8_t* dst = sStage + st * C::kTileBytes;
-          for (int a = 0; a < D / 64; ++a)
-            tma_load_3d(smem_u32(dst + a * kTile * 128), part == 0 ? &mkh : &mkl, fb, a * 64, kvh, c * kTile);
+          for (int a = 0; a < D / 64; ++a) {
+            const uint32_t da = smem_u32(dst + a * kTile * 128);
+            if (k_mode == 0)
+              tma_load_3d(da, part == 0 ? &mkh : &mkl, fb, a * 64, kvh, c * kTile);
+            else if (k_mode == 1)
+              tma_load_4d(da, &mkh, fb, a * 64, kvh, h % S, c * kTile);
+            else
+              tma_load_3d(da, &mkh, fb, a * 64, h, c * kTile);
+          }
           ++k;
         }
       }
@@ -143,24 +160,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = wait_bar(smem_u32(&ctl->q_full), 0, guard, 2);
-      tc_fence_after();
+      // descriptor bases (K-major, 128-byte swizzle), stepped with 32-bit adds
+      const uint32_t q_lo = sdesc_sw128_lo(smem_u32(sQ), 16);
+      const uint32_t k_lo = sdesc_sw128_lo(smem_u32(sStage), 16);
+      constexpr uint32_t d_hi = sdesc_sw128_hi(1024);
       int k = 0;
       for (int n = 0; n < n_seq && ok; ++n) {
         const int b = n & 1;
         if (!wait_bar(smem_u32(&ctl->s_empty[b]), ((n >> 1) & 1) ^ 1, guard, 3)) { ok = false; break; }
         tc_fence_after();
         const uint32_t dcol = tm + b * kTile;
-        for (int part = 0; part < 2; ++part) {
+        for (int part = 0; part < parts; ++part) {
           const int st = k % C::kStages;
           if (!wait_bar(smem_u32(&ctl->full[st]), (k / C::kStages) & 1, guard, 4)) { ok = false; break; }
-          tc_fence_after();
-          const uint8_t* kt = sStage + st * C::kTileBytes;
+          const uint32_t kb = k_lo + st * (C::kTileBytes >> 4);
 #pragma unroll
-          for (int kk = 0; kk < KSTEPS; ++kk) {
-            const uint64_t ad = sdesc_sw128(smem_u32(sQ + (kk >> 2) * kTile * 128 + 32 * (kk & 3)), 16, 1024);
-            const uint64_t bd = sdesc_sw128(smem_u32(kt + (kk >> 2) * kTile * 128 + 32 * (kk & 3)), 16, 1024);
-            umma_ss(dcol, ad, bd, kIdesc, (part > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < KSTEPS; ++kk)
+            umma_ss_lh(dcol, q_lo + (kk >> 2) * (kTile * 128 >> 4) + 2 * (kk & 3), d_hi,
+                       kb + (kk >> 2) * (kTile * 128 >> 4) + 2 * (kk & 3), d_hi, kIdesc,
+                       (part > 0 || kk > 0) ? 1u : 0u);
           umma_commit(smem_u32(&ctl->empty[st]));
           ++k;
         }
@@ -268,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 template <int D, int LOGR>
 cudaError_t launch_search_t(const CUtensorMap& mqs, const CUtensorMap& mkh, const CUtensorMap& mkl, float* mass,
-                            int H, int Hkv, int S, int Ns, int Nb, float sl2, const DeviceGuardArgs& g,
-                            cudaStream_t stream) {
+                            int H, int Hkv, int S, int Ns, int Nb, float sl2, int q_mode, int k_mode,
+                            const DeviceGuardArgs& g, cudaStream_t stream) {
   using C = SearchCfg<D>;
   static bool attr = false;
   if (!attr) {
@@ -280,40 +298,51 @@ cudaError_t launch_search_t(const CUtensorMap& mqs, const CUtensorMap& mkh, cons
   }
   const int n_row_tiles = (Ns + kTile - 1) / kTile;
   search_kernel<D, LOGR><<<static_cast<unsigned>(n_row_tiles) * H, kThreads, C::kSmem, stream>>>(
-      mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, g.status, g.limit_ns);
+      mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, q_mode, k_mode, g.status, g.limit_ns);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t dispatch_r(int logr, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, float* mass,
-                       int H, int Hkv, int S, int Ns, int Nb, float sl2, const DeviceGuardArgs& g, cudaStream_t st) {
+                       int H, int Hkv, int S, int Ns, int Nb, float sl2, int qm, int km, const DeviceGuardArgs& g,
+                       cudaStream_t st) {
   switch (logr) {
-    case 0: return launch_search_t<D, 0>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
-    case 1: return launch_search_t<D, 1>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
-    case 2: return launch_search_t<D, 2>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
-    case 3: return launch_search_t<D, 3>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
-    case 4: return launch_search_t<D, 4>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
-    case 5: return launch_search_t<D, 5>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
-    case 6: return launch_search_t<D, 6>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
-    case 7: return launch_search_t<D, 7>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, g, st);
+    case 0: return launch_search_t<D, 0>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
+    case 1: return launch_search_t<D, 1>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
+    case 2: return launch_search_t<D, 2>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
+    case 3: return launch_search_t<D, 3>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
+    case 4: return launch_search_t<D, 4>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
+    case 5: return launch_search_t<D, 5>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
+    case 6: return launch_search_t<D, 6>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
+    case 7: return launch_search_t<D, 7>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 }  // namespace
 
-cudaError_t launch_search(const void* q, const void* khi, const void* klo, float* mass, int L, int H, int Hkv,
-                          int d, int B, int S, const DeviceGuardArgs& g, cudaStream_t stream) {
+cudaError_t launch_search(const SearchSources& src, float* mass, int L, int H, int Hkv, int d, int B, int S,
+                          const DeviceGuardArgs& g, cudaStream_t stream) {
   const int Ns = L / S, Nb = L / B, r = B / S;
   int logr = 0;
   while ((1 << logr) < r) ++logr;
   CUtensorMap mqs, mkh, mkl;
-  if (!make_tmap_sampled(&mqs, q, L, H, d, S, kTile) || !make_tmap_rows(&mkh, khi, Ns, Hkv, d, kTile) ||
-      !make_tmap_rows(&mkl, klo, Ns, Hkv, d, kTile))
-    return cudaErrorInvalidValue;
+  bool ok = src.q_mode == 0 ? make_tmap_sampled(&mqs, src.q, L, H, d, S, kTile)
+                            : make_tmap_rows(&mqs, src.q, Ns, H, d, kTile);
+  if (src.k_mode == 0) {
+    ok = ok && make_tmap_rows(&mkh, src.k_a, Ns, Hkv, d, kTile) && make_tmap_rows(&mkl, src.k_b, Ns, Hkv, d, kTile);
+  } else if (src.k_mode == 1) {
+    ok = ok && make_tmap_sampled(&mkh, src.k_a, L, Hkv, d, S, kTile);
+    mkl = mkh;
+  } else {
+    ok = ok && make_tmap_rows(&mkh, src.k_a, Ns, H, d, kTile);
+    mkl = mkh;
+  }
+  if (!ok) return cudaErrorInvalidValue;
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
-  if (d == 128) return dispatch_r<128>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, g, stream);
-  return dispatch_r<64>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, g, stream);
+  if (d == 128)
+    return dispatch_r<128>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, src.q_mode, src.k_mode, g, stream);
+  return dispatch_r<64>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, src.q_mode, src.k_mode, g, stream);
 }
 
 }  // namespace rr

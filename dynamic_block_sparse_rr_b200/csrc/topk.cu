@@ -50,7 +50,7 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T* warp_buf, T* total) {
 
 __global__ void __launch_bounds__(kThreads) top_tau_kernel(const float* __restrict__ mass, int H, int Nb,
                                                            float tau, int32_t* __restrict__ count,
-                                                           int32_t* __restrict__ idx, int p2max) {
+                                                           int32_t* __restrict__ idx, int p2max, int rep) {
   extern __shared__ __align__(16) uint8_t smem[];
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem);
   unsigned char* sel = reinterpret_cast<unsigned char*>(keys + p2max);
@@ -63,12 +63,16 @@ __global__ void __launch_bounds__(kThreads) top_tau_kernel(const float* __restri
   const int h = static_cast<int>(blockIdx.x % H);
   const long long row = static_cast<long long>(h) * Nb + I;
   const int n = I + 1;
-  int32_t* out = idx + row * Nb;
+  // output rows: heads h*rep .. h*rep+rep-1 (rep > 1: one mask for a GQA group)
+  const long long orow = static_cast<long long>(h) * rep * Nb + I;
+  const long long ostride = static_cast<long long>(Nb) * Nb;   // between output heads
+  int32_t* out = idx + orow * Nb;
   const int tid = threadIdx.x;
 
   if (I == Nb - 1 || !(tau < 1.0f)) {  // protected last row, or tau >= 1: every causal block
-    for (int t = tid; t < n; t += kThreads) out[t] = t;
-    if (tid == 0) count[row] = n;
+    for (int r = 0; r < rep; ++r)
+      for (int t = tid; t < n; t += kThreads) out[r * ostride + t] = t;
+    if (tid < rep) count[orow + static_cast<long long>(tid) * Nb] = n;
     return;
   }
 
@@ -134,13 +138,16 @@ __global__ void __launch_bounds__(kThreads) top_tau_kernel(const float* __restri
   int tot;
   int pos = block_exclusive_scan<int>(flags, ibuf, &tot);
   for (int t = q0; t < q1; ++t)
-    if (sel[t]) out[pos++] = t;
-  if (tid == 0) count[row] = cnt;
+    if (sel[t]) {
+      for (int r = 0; r < rep; ++r) out[r * ostride + pos] = t;
+      ++pos;
+    }
+  if (tid < rep) count[orow + static_cast<long long>(tid) * Nb] = cnt;
 }
 
 }  // namespace
 
-cudaError_t launch_top_tau(const float* mass, int H, int Nb, float tau, int32_t* count, int32_t* idx,
+cudaError_t launch_top_tau(const float* mass, int H, int Nb, float tau, int32_t* count, int32_t* idx, int rep,
                            cudaStream_t stream) {
   if (H <= 0 || Nb <= 0) return cudaSuccess;
   int p2 = 1;
@@ -153,7 +160,7 @@ cudaError_t launch_top_tau(const float* mass, int H, int Nb, float tau, int32_t*
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  top_tau_kernel<<<static_cast<unsigned>(H) * Nb, kThreads, smem, stream>>>(mass, H, Nb, tau, count, idx, p2);
+  top_tau_kernel<<<static_cast<unsigned>(H) * Nb, kThreads, smem, stream>>>(mass, H, Nb, tau, count, idx, p2, rep);
   return cudaGetLastError();
 }
 

@@ -74,6 +74,35 @@ rr_status rr_search(const void* q, const void* k, int L, int H, int Hkv, int d, 
                     float tau, int32_t* count, int32_t* idx, float* mass, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* Sampling variants of the pattern search.  The pages fix the head rotation of
+ * the sampled offset and the stride-level aggregation of keys, but leave open
+ * three choices, each selectable here (flags may be combined; 0 = rr_search):
+ *   RR_VAR_ROTATE        the offset rotates across strides as well as heads:
+ *                        head h samples, in stride i, the query at
+ *                        i*S + ((h + i) mod S).
+ *   RR_VAR_SAMPLED_KEYS  the key side of stride j is the single key at the
+ *                        head's own sampled position of that stride (the same
+ *                        rule as its queries) instead of the mean of the S
+ *                        keys: same O(L^2/S^2) cost, no averaging.
+ *   RR_VAR_GQA_MASK      one mask per GQA group: the Top-tau selection runs
+ *                        on the sum of the block masses of the H/Hkv query
+ *                        heads of a kv head, and every head of the group
+ *                        receives that selection (rows of count/idx repeat).
+ * Scores, block mass, Top-tau and the last-row protection are those of
+ * rr_search.  Out: count [H,Nb], idx [H,Nb,Nb]; mass (optional) receives the
+ * per-head block mass [H,Nb,Nb] before any group sum.  The workspace is sized
+ * by rr_workspace_size_variant with the same flags (it holds the gathered
+ * rows [L/S, H, d] bf16 when rotating, the group masses [Hkv, Nb, Nb] fp32
+ * with RR_VAR_GQA_MASK).  Unknown flag bits: RR_EINVAL. */
+#define RR_VAR_ROTATE 1u
+#define RR_VAR_SAMPLED_KEYS 2u
+#define RR_VAR_GQA_MASK 4u
+rr_status rr_workspace_size_variant(int L, int H, int Hkv, int d, int B, int S, unsigned flags,
+                                    size_t* bytes);
+rr_status rr_search_variant(const void* q, const void* k, int L, int H, int Hkv, int d, int B, int S,
+                            float tau, unsigned flags, int32_t* count, int32_t* idx, float* mass,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* Causal block-sparse attention over a block mask (Abstract: "computing only
  * half of the attention blocks"; Figure 2 stage 3).  Query q of block I, head
  * h, attends with scale 1/sqrt(d) to every key k <= q of the blocks listed for

@@ -38,6 +38,13 @@ R7  Static protection of the last query block (TL;DR): the last row I = Nb-1
 R8  Block-sparse causal attention ("computing only half of the attention
     blocks").  Query q in block I attends, with softmax scale 1/sqrt(d), to
     every key k <= q that lies in a selected block of row I.
+V1-V3 Variants the pages leave open (off by default): V1 rotates the sampled
+    offset across strides too, p(h, i) = i*S + ((h + i) mod S); V2 takes the key
+    side of stride j as the single key at the head's offset instead of the
+    stride mean (same O(L^2/S^2) cost, no blurring of per-token structure); V3
+    keeps one mask per GQA group, selecting on the summed block mass of the
+    group's heads.                                            [parity unpinned
+    beyond the invariants in tests/test_oracle.py]
 R9  Mask comparison band (tolerance of the operator's specification): a block
     is near-threshold when the running sum just before or just after it, in
     the R6 order, lies within `band` of tau; a near-tie is a pair of blocks at
@@ -70,6 +77,14 @@ def sampled_positions(L: int, H: int, S: int) -> np.ndarray:
     return np.stack([i * S + (h % S) for h in range(H)])
 
 
+def rotated_positions(L: int, H: int, S: int) -> np.ndarray:
+    """Variant V1 (rotation across strides as well as heads): head h samples, in
+    stride i, the query at i*S + ((h + i) mod S).  Shape [H, L/S]."""
+    Ns = L // S
+    i = np.arange(Ns, dtype=np.int64)
+    return np.stack([i * S + (h + i) % S for h in range(H)])
+
+
 # ------------------------------------------------------------ R2 stride keys
 def pool_keys(K: np.ndarray, S: int) -> np.ndarray:
     """Kbar[j, kv, :] = mean over the S keys of stride j (R2).  K: [L, Hkv, d]."""
@@ -78,23 +93,30 @@ def pool_keys(K: np.ndarray, S: int) -> np.ndarray:
 
 
 # ------------------------------------------------------- R3-R5 block masses
-def block_mass(Q: np.ndarray, K: np.ndarray, B: int, S: int, row_chunk: int = 2048) -> np.ndarray:
+def block_mass(Q: np.ndarray, K: np.ndarray, B: int, S: int, row_chunk: int = 2048,
+               rotate: bool = False, sampled_keys: bool = False) -> np.ndarray:
     """Unnormalised block mass M[h, I, J] (R3-R5), zero above the diagonal.
 
-    Q: [L, H, d], K: [L, Hkv, d] (float64).  Returns [H, Nb, Nb] float64.
+    Q: [L, H, d], K: [L, Hkv, d].  Returns [H, Nb, Nb] float64.
+    Variants (off by default): rotate -> V1 query positions; sampled_keys -> V2,
+    the key side of stride j is the single key at the head's own offset in that
+    stride (the same rule as its queries) instead of the stride mean.
     """
     L, H, d = Q.shape
     Hkv = K.shape[1]
     g = H // Hkv
     Ns, Nb, r = L // S, L // B, B // S
-    Kbar = pool_keys(K, S)
-    pos = sampled_positions(L, H, S)
+    Kbar = None if sampled_keys else pool_keys(K, S)
+    pos = rotated_positions(L, H, S) if rotate else sampled_positions(L, H, S)
     scale = 1.0 / math.sqrt(d)
     M = np.zeros((H, Nb, Nb), dtype=np.float64)
     step = max(r, (row_chunk // r) * r)
     for h in range(H):
         Qs = Q[pos[h], h, :].astype(np.float64)  # [Ns, d] real sampled queries
-        Kb = Kbar[:, h // g, :]                  # [Ns, d]
+        if sampled_keys:
+            Kb = K[pos[h], h // g, :].astype(np.float64)   # [Ns, d] one real key per stride
+        else:
+            Kb = Kbar[:, h // g, :]                  # [Ns, d]
         for a in range(0, Ns, step):
             b = min(Ns, a + step)
             s = (Qs[a:b] @ Kb[:b].T) * scale     # rows i in [a,b), strides j < b
@@ -107,6 +129,15 @@ def block_mass(Q: np.ndarray, K: np.ndarray, B: int, S: int, row_chunk: int = 20
             nI, nJ = (b - a) // r, b // r
             M[h, a // r:a // r + nI, :nJ] += P.reshape(nI, r, nJ, r).sum(axis=(1, 3))
     return M
+
+
+def group_mass(M: np.ndarray, Hkv: int) -> np.ndarray:
+    """Variant V3 (one mask per GQA group): the block masses of the g query heads
+    of each kv head summed, repeated for every head of the group.  [H, Nb, Nb]."""
+    H, Nb, _ = M.shape
+    g = H // Hkv
+    Mg = M.reshape(Hkv, g, Nb, Nb).sum(axis=1)
+    return np.repeat(Mg, g, axis=0)
 
 
 def normalise_mass(M: np.ndarray) -> np.ndarray:
@@ -149,9 +180,14 @@ def select(m: np.ndarray, tau: float):
     return count, idx
 
 
-def rr_search(Q: np.ndarray, K: np.ndarray, B: int, S: int, tau: float):
-    """The pattern search: returns (count, idx, m) with m the normalised block mass."""
-    m = normalise_mass(block_mass(Q, K, B, S))
+def rr_search(Q: np.ndarray, K: np.ndarray, B: int, S: int, tau: float, rotate: bool = False,
+              sampled_keys: bool = False, gqa_mask: bool = False):
+    """The pattern search: returns (count, idx, m) with m the normalised block mass
+    (of the GQA group when gqa_mask)."""
+    M = block_mass(Q, K, B, S, rotate=rotate, sampled_keys=sampled_keys)
+    if gqa_mask:
+        M = group_mass(M, K.shape[1])
+    m = normalise_mass(M)
     count, idx = select(m, tau)
     return count, idx, m
 

@@ -119,3 +119,44 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(m, "_lib", None)
     with pytest.raises(ImportError):
         m.lib()
+
+
+def _ws_var(L, H, Hkv, d, B, S, flags):
+    n = ctypes.c_size_t()
+    code = rr_lib().rr_workspace_size_variant(L, H, Hkv, d, B, S, flags, ctypes.byref(n))
+    return code, n.value
+
+
+def test_variant_workspace_sizes(rr):
+    L, H, Hkv, d, B, S = 4096, 8, 2, 128, 128, 16
+    Ns, Nb = L // S, L // B
+    assert _ws_var(L, H, Hkv, d, B, S, 0) == _ws(L, H, Hkv, d, B, S)
+    base = _ws_var(L, H, Hkv, d, B, S, 0)[1]
+    # sampled keys drop the pooled (hi, lo) pair
+    assert _ws_var(L, H, Hkv, d, B, S, rr.VAR_SAMPLED_KEYS)[1] == base - 2 * Ns * Hkv * d * 2
+    # rotation adds the gathered queries, and the gathered keys with sampled keys
+    assert _ws_var(L, H, Hkv, d, B, S, rr.VAR_ROTATE)[1] == base + Ns * H * d * 2
+    assert (_ws_var(L, H, Hkv, d, B, S, rr.VAR_ROTATE | rr.VAR_SAMPLED_KEYS)[1]
+            == base - 2 * Ns * Hkv * d * 2 + 2 * Ns * H * d * 2)
+    # the GQA mask adds the group masses
+    assert _ws_var(L, H, Hkv, d, B, S, rr.VAR_GQA_MASK)[1] == base + Hkv * Nb * Nb * 4
+    assert _ws_var(L, H, Hkv, d, B, S, 8)[0] == rr.RR_EINVAL
+    assert _ws_var(L, H, Hkv, d, B, 3, 1)[0] == rr.RR_EINVAL
+
+
+def test_search_variant_rejects_before_any_launch(rr):
+    lib = rr.lib()
+    g = 1 << 20
+    L, H, Hkv, d, B, S = 1024, 4, 2, 64, 64, 4
+    flags = rr.VAR_ROTATE | rr.VAR_SAMPLED_KEYS | rr.VAR_GQA_MASK
+    _, n = _ws_var(L, H, Hkv, d, B, S, flags)
+
+    def call(flags=flags, q=g, nws=n, tau=0.9):
+        return lib.rr_search_variant(q, g, L, H, Hkv, d, B, S, tau, flags, g, g, None, g, nws, None)
+
+    assert call(flags=16) == rr.RR_EINVAL
+    assert call(q=None) == rr.RR_EINVAL
+    assert call(q=g + 2) == rr.RR_EALIGN
+    assert call(tau=0.0) == rr.RR_EINVAL
+    assert call(nws=n - 1) == rr.RR_EINVAL           # the variant workspace is larger than the plain one
+    assert n > _ws(L, H, Hkv, d, B, S)[1]

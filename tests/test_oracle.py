@@ -317,3 +317,60 @@ def test_recall_of_single_block_equals_its_exact_share():
     for I in range(4):
         want = A[I * B:(I + 1) * B, 0:B].sum() / B
         assert abs(rec[0, I] - want) < 1e-12
+
+
+# ------------------------------------------------------------ sampling variants
+@pytest.mark.parametrize("L,H,S", [(1024, 4, 4), (4096, 32, 16), (512, 3, 8)])
+def test_rotated_positions_rotate_across_strides(L, H, S):
+    p = oracle.rotated_positions(L, H, S)
+    Ns = L // S
+    i = np.arange(Ns)
+    for h in range(H):
+        off = p[h] - i * S
+        assert np.all((off >= 0) & (off < S))
+        assert np.array_equal(off, (h + i) % S)
+        # over S consecutive strides every head visits every offset once
+        for a in range(0, Ns - S + 1, S):
+            assert sorted(off[a:a + S].tolist()) == list(range(S))
+    if H >= S:
+        for i0 in range(min(Ns, 8)):
+            assert sorted((p[:S, i0] - i0 * S).tolist()) == list(range(S))
+
+
+def test_sampled_keys_equal_mean_keys_when_strides_are_constant():
+    L, H, Hkv, d, B, S = 256, 4, 2, 16, 32, 4
+    Q = _rand((L, H, d), 60)
+    K = np.repeat(_rand((L // S, Hkv, d), 61), S, axis=0)       # keys constant inside each stride
+    for rotate in (False, True):
+        a = oracle.block_mass(Q, K, B, S, rotate=rotate)
+        b = oracle.block_mass(Q, K, B, S, rotate=rotate, sampled_keys=True)
+        assert np.max(np.abs(a - b)) < 1e-12
+
+
+def test_variants_at_stride_one_are_exact():
+    L, H, Hkv, d, B = 256, 2, 1, 16, 32
+    Q, K = _rand((L, H, d), 62), _rand((L, Hkv, d), 63)
+    ref = oracle.block_mass(Q, K, B, 1)
+    for rotate in (False, True):
+        for sk in (False, True):
+            assert np.max(np.abs(oracle.block_mass(Q, K, B, 1, rotate=rotate, sampled_keys=sk) - ref)) < 1e-12
+
+
+def test_gqa_group_mask_shares_lists_and_reaches_tau():
+    L, H, Hkv, d, B, S, tau = 512, 4, 2, 16, 32, 4, 0.9
+    Q, K = _rand((L, H, d), 64), _rand((L, Hkv, d), 65)
+    count, idx, m = oracle.rr_search(Q, K, B, S, tau, gqa_mask=True)
+    M = oracle.block_mass(Q, K, B, S)
+    Mg = M[0] + M[1]
+    assert np.allclose(oracle.normalise_mass(Mg[None])[0], m[0], atol=1e-14)
+    Nb = L // B
+    for kv in range(Hkv):
+        for h in (2 * kv, 2 * kv + 1):
+            assert np.array_equal(count[h], count[2 * kv])
+            for I in range(Nb):
+                assert np.array_equal(idx[h, I, :count[h, I]], idx[2 * kv, I, :count[2 * kv, I]])
+        for I in range(Nb - 1):
+            assert m[2 * kv, I, idx[2 * kv, I, :count[2 * kv, I]]].sum() >= tau - 1e-12
+    c1, i1, _ = oracle.rr_search(Q, K.repeat(2, axis=1), B, S, tau, gqa_mask=True)   # g = 1: per-head masks
+    c2, i2, _ = oracle.rr_search(Q, K.repeat(2, axis=1), B, S, tau)
+    assert np.array_equal(c1, c2)

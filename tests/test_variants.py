@@ -1,0 +1,115 @@
+"""Parity of the search's sampling variants (rr_search_variant) against the oracle.
+
+V1 rotates the sampled offset across strides, V2 replaces the stride mean of the
+keys by the key at the head's own sampled position, V3 selects one mask per GQA
+group from the group's summed block mass; any combination.  The per-head block
+mass must agree with the oracle's within the same bound as the plain search, the
+mask within the near-threshold band, and every head of a GQA group must carry
+the same mask.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gen
+import oracle
+from tests.mask_compare import check_mask_format, compare_masks
+
+pytestmark = pytest.mark.gpu
+
+MASS_ERR = 2e-5
+
+ROT, SK, GQA = 1, 2, 4
+ALL_FLAGS = [0, ROT, SK, ROT | SK, GQA, ROT | GQA, SK | GQA, ROT | SK | GQA]
+
+
+@pytest.fixture(scope="module")
+def rr():
+    from dynamic_block_sparse_rr_b200 import _build
+    _build.build()
+    import dynamic_block_sparse_rr_b200 as m
+    assert torch.cuda.is_available(), "the variant parity tests need a CUDA device"
+    m.lib()
+    return m
+
+
+def to_dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def run_case(rr, L, H, Hkv, d, B, S, tau, flags, structure, seed):
+    q, k, _ = gen.make_qkv(L, H, Hkv, d, structure, seed)
+    Q, K = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k)
+    qd, kd = to_dev(q), to_dev(k)
+    Nb = L // B
+    mass = torch.zeros((H, Nb, Nb), dtype=torch.float32, device="cuda")
+    ws = rr.workspace(L, H, Hkv, d, B, S, flags=flags)
+    count, idx = rr.search_variant(qd, kd, B, S, tau, flags, mass=mass, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+    torch.cuda.synchronize()
+    count, idx = count.cpu().numpy(), idx.cpu().numpy()
+    M_g = mass.cpu().numpy().astype(np.float64)
+    rot, sk, gqa = bool(flags & ROT), bool(flags & SK), bool(flags & GQA)
+
+    check_mask_format(count, idx)
+    M_o = oracle.block_mass(Q, K, B, S, rotate=rot, sampled_keys=sk)
+    tri = np.tri(Nb, dtype=bool)[None]
+    err = float(np.max(np.abs(np.where(tri, oracle.normalise_mass(M_g) - oracle.normalise_mass(M_o), 0.0))))
+    assert err <= MASS_ERR, f"per-head block mass error {err} (flags {flags})"
+    count_o, idx_o, m_o = oracle.rr_search(Q, K, B, S, tau, rotate=rot, sampled_keys=sk, gqa_mask=gqa)
+    st = compare_masks(count, idx, count_o, idx_o, m_o, tau)
+    assert st["blocks_fail"] == 0, (flags, st)
+    if gqa:
+        g = H // Hkv
+        for kv in range(Hkv):
+            for t in range(1, g):
+                assert np.array_equal(count[kv * g + t], count[kv * g]), (flags, kv, t)
+                for I in range(Nb):
+                    c = count[kv * g, I]
+                    assert np.array_equal(idx[kv * g + t, I, :c], idx[kv * g, I, :c])
+    return count, idx, st
+
+
+@pytest.mark.parametrize("flags", ALL_FLAGS)
+def test_variant_flags(rr, flags):
+    run_case(rr, 2048, 8, 2, 128, 128, 16, 0.9, flags, gen.PLANTED, seed=21)
+
+
+@pytest.mark.parametrize("L,H,Hkv,d,B,S,tau,structure", [
+    (1600, 4, 2, 64, 64, 4, 0.9, gen.PLANTED),        # ragged sampled-row tile (Ns = 400)
+    (4096, 7, 1, 128, 128, 16, 0.95, gen.VIDEO),     # GQA 7:1, video-like frames
+    (2240, 4, 4, 128, 64, 8, 0.9, gen.PLANTED_BAND),  # Nb = 35 (no float4 group sums needed)
+    (512, 3, 3, 64, 64, 64, 0.5, gen.IID),           # r = 1
+])
+def test_variants_shapes(rr, L, H, Hkv, d, B, S, tau, structure):
+    for flags in (ROT | SK, ROT | SK | GQA, SK):
+        run_case(rr, L, H, Hkv, d, B, S, tau, flags, structure, seed=22)
+
+
+def test_variants_reduce_to_plain_search_at_stride_one(rr):
+    """At S = 1 every query is sampled and each stride is one key: rotation and
+    sampled keys change nothing, so the masks equal the plain search's."""
+    L, H, Hkv, d, B = 1024, 4, 2, 64, 64
+    q, k, _ = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 23)
+    qd, kd = to_dev(q), to_dev(k)
+    c0, i0 = rr.search(qd, kd, B, 1, 0.9)
+    c1, i1 = rr.search_variant(qd, kd, B, 1, 0.9, ROT | SK)
+    torch.cuda.synchronize()
+    assert torch.equal(c0, c1)
+    Nb = L // B
+    cols = torch.arange(Nb, device="cuda")[None, None, :] < c0[:, :, None]
+    assert torch.equal(torch.where(cols, i0, 0), torch.where(cols, i1, 0))
+
+
+def test_flags_zero_is_rr_search(rr):
+    """rr_search_variant with flags 0 returns rr_search's mask bit for bit."""
+    L, H, Hkv, d, B, S = 2048, 4, 2, 128, 128, 16
+    q, k, _ = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 24)
+    qd, kd = to_dev(q), to_dev(k)
+    c0, i0 = rr.search(qd, kd, B, S, 0.9)
+    c1, i1 = rr.search_variant(qd, kd, B, S, 0.9, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(c0, c1)
+    Nb = L // B
+    cols = torch.arange(Nb, device="cuda")[None, None, :] < c0[:, :, None]
+    assert torch.equal(torch.where(cols, i0, 0), torch.where(cols, i1, 0))
