@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(kThreads) top_tau_kernel(const float* __restri
   if (I == Nb - 1 || !(tau < 1.0f)) {  // protected last row, or tau >= 1: every causal block
     for (int r = 0; r < rep; ++r)
       for (int t = tid; t < n; t += kThreads) out[r * ostride + t] = t;
-    if (tid < rep) count[orow + static_cast<long long>(tid) * Nb] = n;
+    for (int r = tid; r < rep; r += kThreads) count[orow + static_cast<long long>(r) * Nb] = n;
     return;
   }
 
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kThreads) top_tau_kernel(const float* __restri
       for (int r = 0; r < rep; ++r) out[r * ostride + pos] = t;
       ++pos;
     }
-  if (tid < rep) count[orow + static_cast<long long>(tid) * Nb] = cnt;
+  for (int r = tid; r < rep; r += kThreads) count[orow + static_cast<long long>(r) * Nb] = cnt;
 }
 
 }  // namespace
