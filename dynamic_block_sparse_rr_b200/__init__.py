@@ -23,7 +23,7 @@ RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT, RR_ESCRATCH
 # every symbol that include/rr.h declares
 EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status",
            "rr_set_wait_limit_ns", "rr_status_string", "rr_search_static", "rr_mask_recall",
-           "rr_workspace_size_variant", "rr_search_variant")
+           "rr_workspace_size_variant", "rr_search_variant", "rr_mask_to_dense")
 
 # sampling-variant flags of rr_search_variant (rr.h)
 VAR_ROTATE, VAR_SAMPLED_KEYS, VAR_GQA_MASK = 1, 2, 4
@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.rr_workspace_size_variant.restype = ctypes.c_int
         L.rr_search_variant.argtypes = [vp, vp, i, i, i, i, i, i, f, u, vp, vp, vp, vp, sz, vp]
         L.rr_search_variant.restype = ctypes.c_int
+        L.rr_mask_to_dense.argtypes = [vp, vp, i, i, vp, vp]
+        L.rr_mask_to_dense.restype = ctypes.c_int
         L.rr_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.rr_set_wait_limit_ns.restype = ctypes.c_uint64
         L.rr_status_string.argtypes = [i]
@@ -217,3 +219,13 @@ def check_status(ws, stream=None) -> int:
 
 def set_wait_limit_ns(ns: int) -> int:
     return lib().rr_set_wait_limit_ns(int(ns))
+
+
+def mask_to_dense(count, idx, out=None, stream=None):
+    """Dense uint8 view [H, Nb, Nb] of a block mask (1 where a block is listed)."""
+    H, Nb = count.shape
+    if out is None:
+        out = torch.empty((H, Nb, Nb), dtype=torch.uint8, device=count.device)
+    _check(lib().rr_mask_to_dense(count.data_ptr(), idx.data_ptr(), H, Nb, out.data_ptr(), _stream(stream)),
+           "rr_mask_to_dense")
+    return out

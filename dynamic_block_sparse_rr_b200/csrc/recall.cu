@@ -1,5 +1,5 @@
-// recall.cu — mask diagnostics: the share of a row's exact attention mass that a
-// block mask keeps (the synthetic analogue of RRAttention's pattern
+// recall.cu — mask diagnostics: the dense view of a block mask, and the share
+// of a row's exact attention mass that a block mask keeps (the synthetic analogue of RRAttention's pattern
 // visualisations, sciencestack page, Figures 4 and 5: full-attention ground
 // truth against the RR selection).
 //
@@ -43,7 +43,36 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   if (lane == 0) recall[row] = tot > 0.0 ? static_cast<float>(kept / tot) : 0.0f;
 }
 
+// Dense view of a block mask: one warp per (h, I) row clears the row's Nb bytes,
+// then sets dense[h, I, J] = 1 for each listed J in [0, Nb).
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    mask_to_dense_kernel(const int32_t* __restrict__ count, const int32_t* __restrict__ idx, int H, int Nb,
+                         uint8_t* __restrict__ dense) {
+  const long long row = static_cast<long long>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(H) * Nb) return;
+  uint8_t* out = dense + row * Nb;
+  for (int J = lane; J < Nb; J += 32) out[J] = 0;
+  __syncwarp();
+  const int32_t* list = idx + row * Nb;
+  int c = count[row];
+  c = c < 0 ? 0 : (c > Nb ? Nb : c);
+  for (int t = lane; t < c; t += 32) {
+    const int J = list[t];
+    if (J >= 0 && J < Nb) out[J] = 1;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int Nb, uint8_t* dense,
+                                 cudaStream_t stream) {
+  const long long rows = static_cast<long long>(H) * Nb;
+  if (rows == 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>((rows + kWarpsPerBlock - 1) / kWarpsPerBlock);
+  mask_to_dense_kernel<<<blocks, kWarpsPerBlock * 32, 0, stream>>>(count, idx, H, Nb, dense);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_mask_recall(const float* mass, const int32_t* count, const int32_t* idx, int H, int Nb,
                                float* recall, cudaStream_t stream) {

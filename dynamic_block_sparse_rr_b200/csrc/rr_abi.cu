@@ -183,6 +183,15 @@ rr_status rr_mask_recall(const float* mass, const int32_t* count, const int32_t*
   return RR_OK;
 }
 
+rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int Nb, uint8_t* dense, void* stream) {
+  if (!count || !idx || !dense || H <= 0 || Nb <= 0) return RR_EINVAL;
+  if (Nb > rr::kMaxBlocks) return RR_EUNSUPPORTED;
+  if (!aligned16(count) || !aligned16(idx)) return RR_EALIGN;
+  if (rr::launch_mask_to_dense(count, idx, H, Nb, dense, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RR_ECUDA;
+  return RR_OK;
+}
+
 rr_status rr_check_status(void* workspace, void* stream) {
   if (!workspace) return RR_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

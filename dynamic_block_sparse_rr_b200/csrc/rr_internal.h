@@ -52,6 +52,10 @@ cudaError_t launch_bsfa(const void* q, const void* k, const void* v, const int32
                         const int32_t* idx, void* o, int L, int H, int Hkv, int d, int B,
                         const DeviceGuardArgs& g, cudaStream_t stream);
 
+// Dense uint8 view [H, Nb, Nb] of a block mask (diagnostics).
+cudaError_t launch_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int Nb, uint8_t* dense,
+                                 cudaStream_t stream);
+
 // Share of each row's block mass kept by a mask (diagnostics).
 cudaError_t launch_mask_recall(const float* mass, const int32_t* count, const int32_t* idx, int H, int Nb,
                                float* recall, cudaStream_t stream);

@@ -132,6 +132,14 @@ rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H
 rr_status rr_mask_recall(const float* mass, const int32_t* count, const int32_t* idx, int H, int Nb,
                          float* recall, void* stream);
 
+/* Dense view of a block mask (debugging and plotting): dense[(h*Nb + I)*Nb + J]
+ * = 1 when J is among the first count[h*Nb+I] entries of row (h, I) of idx,
+ * else 0.  count [H,Nb] and idx [H,Nb,Nb] int32 as produced by rr_search;
+ * dense [H,Nb,Nb] uint8; all device memory, caller-owned.  Entries outside
+ * [0, Nb) are ignored, count is clamped to [0, Nb].  Asynchronous on `stream`. */
+rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int Nb, uint8_t* dense,
+                           void* stream);
+
 /* Synchronises `stream`, returns the device-side status recorded since the
  * last rr_* call that started on this workspace (RR_OK or RR_ETIMEOUT), and
  * RR_ECUDA if the stream reports an error. */

@@ -284,3 +284,25 @@ def test_mask_recall_matches_oracle(rr, L, H, Hkv, d, B, S, tau):
     rec_o = oracle.mask_recall(M_o, count.cpu().numpy(), idx.cpu().numpy())
     assert np.max(np.abs(rec - rec_o)) <= 1e-5
     assert np.all(rec[:, -1] > 1 - 1e-6)
+
+
+def test_mask_to_dense_matches_lists(rr):
+    """rr_mask_to_dense marks exactly the listed blocks, for a searched mask and
+    for a hand-made one with gaps, duplicates of nothing and an empty row."""
+    from tests.mask_compare import dense_from_lists
+    L, H, Hkv, d, B, S = 2048, 4, 2, 128, 128, 16
+    q, k, _ = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 14)
+    count, idx = rr.search(to_dev(q), to_dev(k), B, S, 0.8)
+    dense = rr.mask_to_dense(count, idx).cpu().numpy()
+    c, i = count.cpu().numpy(), idx.cpu().numpy()
+    assert np.array_equal(dense.astype(bool), dense_from_lists(c, i))
+    Nb = L // B
+    c2 = np.zeros((H, Nb), np.int32)
+    i2 = np.zeros((H, Nb, Nb), np.int32)
+    for h in range(H):
+        for I in range(Nb):
+            sel = list(range(0, I + 1, h + 1)) if I % 3 else []
+            c2[h, I] = len(sel)
+            i2[h, I, :len(sel)] = sel
+    dense2 = rr.mask_to_dense(torch.from_numpy(c2).cuda(), torch.from_numpy(i2).cuda()).cpu().numpy()
+    assert np.array_equal(dense2.astype(bool), dense_from_lists(c2, i2))
