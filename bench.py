@@ -318,29 +318,33 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
         dense_tflops = block_flops(cfg, dense_blocks) / (dense_ms / 1e3) / 1e12
         del cd, idd
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: rr_attention_host
+    # copies q, k, v in and o out (page-locked host memory) inside the call,
+    # pipelined against the kernels kv head by kv head
     oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(1, min(args.steps, 2))
-    qd2, kd2, vd2 = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws_host = torch.empty(rr.workspace_size_host(L, H, Hkv, d, B, S), dtype=torch.uint8, device=dev)
+    copy_stream = torch.cuda.Stream(device=dev)
+    rr.attention_host(qh, kh, vh, B, S, tau, out=oh, count=count, idx=idx, ws=ws_host, stream=stream,
+                      copy_stream=copy_stream)   # warm-up (first-call setup outside the timed region)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        qd2.copy_(qh, non_blocking=True)
-        kd2.copy_(kh, non_blocking=True)
-        vd2.copy_(vh, non_blocking=True)
-        rr.attention(qd2, kd2, vd2, B, S, tau, out=o, count=count, idx=idx, ws=ws)
-        oh.copy_(o, non_blocking=True)
+        rr.attention_host(qh, kh, vh, B, S, tau, out=oh, count=count, idx=idx, ws=ws_host, stream=stream,
+                          copy_stream=copy_stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if rr.check_status(ws_host) != rr.RR_OK:
+        raise RuntimeError("device-side status after the end-to-end run")
+    del ws_host
     total_ms_max, e2e_ms_max, flops_all = aggregate(total_ms, e2e_ms, flops, world, dev)
     ms_per_step = total_ms_max / args.steps
     value = flops_all / (ms_per_step / 1e3) / 1e12
     e2e_value = flops_all / (e2e_ms_max / 1e3) / 1e12
     h2d = (qh.numel() + kh.numel() + vh.numel()) * 2
     d2h = oh.numel() * 2
-    del qd2, kd2, vd2
 
     peaks = measured_peaks()
     peak = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
@@ -365,7 +369,8 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
             "speedup_vs_dense": (dense_ms / (total_ms / args.steps)) if dense_ms else None,
             "visited_blocks": visited, "visited_fraction": visited / (H * Nb * (Nb + 1) / 2),
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms_max,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "path": "rr_attention_host: pinned host q/k/v/o, copies pipelined per kv head"},
             "gpu_launches": gpu_launches, "clocks": clk, "roofline": roofline, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

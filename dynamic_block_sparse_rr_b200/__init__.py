@@ -23,7 +23,8 @@ RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT, RR_ESCRATCH
 # every symbol that include/rr.h declares
 EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status",
            "rr_set_wait_limit_ns", "rr_status_string", "rr_search_static", "rr_mask_recall",
-           "rr_workspace_size_variant", "rr_search_variant", "rr_mask_to_dense")
+           "rr_workspace_size_variant", "rr_search_variant", "rr_mask_to_dense",
+           "rr_workspace_size_host", "rr_attention_host")
 
 # sampling-variant flags of rr_search_variant (rr.h)
 VAR_ROTATE, VAR_SAMPLED_KEYS, VAR_GQA_MASK = 1, 2, 4
@@ -61,6 +62,10 @@ def lib() -> ctypes.CDLL:
         L.rr_search_variant.argtypes = [vp, vp, i, i, i, i, i, i, f, u, vp, vp, vp, vp, sz, vp]
         L.rr_search_variant.restype = ctypes.c_int
         L.rr_mask_to_dense.argtypes = [vp, vp, i, i, vp, vp]
+        L.rr_workspace_size_host.argtypes = [i, i, i, i, i, i, ctypes.POINTER(sz)]
+        L.rr_workspace_size_host.restype = ctypes.c_int
+        L.rr_attention_host.argtypes = [vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp, vp, sz, vp, vp]
+        L.rr_attention_host.restype = ctypes.c_int
         L.rr_mask_to_dense.restype = ctypes.c_int
         L.rr_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.rr_set_wait_limit_ns.restype = ctypes.c_uint64
@@ -229,3 +234,43 @@ def mask_to_dense(count, idx, out=None, stream=None):
     _check(lib().rr_mask_to_dense(count.data_ptr(), idx.data_ptr(), H, Nb, out.data_ptr(), _stream(stream)),
            "rr_mask_to_dense")
     return out
+
+
+def workspace_size_host(L: int, H: int, Hkv: int, d: int, B: int, S: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().rr_workspace_size_host(L, H, Hkv, d, B, S, ctypes.byref(n)), "rr_workspace_size_host")
+    return n.value
+
+
+_copy_streams = {}
+
+
+def attention_host(qh, kh, vh, B: int, S: int, tau: float, out=None, count=None, idx=None, ws=None,
+                   stream=None, copy_stream=None, device=None):
+    """rr_attention on host tensors (CPU, bf16, contiguous; page-locked for
+    asynchronous copies), copies pipelined against the kernels kv head by kv
+    head -> (o_host, count, idx); the mask stays on the device."""
+    if qh.dim() != 3 or kh.dim() != 3 or vh.shape != kh.shape:
+        raise ValueError("q must be [L, H, d], k and v [L, Hkv, d]")
+    for t in (qh, kh, vh):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 host tensors")
+    L, H, d = qh.shape
+    Hkv = kh.shape[1]
+    Nb = L // B
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if out is None:
+        out = torch.empty(qh.shape, dtype=torch.bfloat16, pin_memory=True)
+    if count is None or idx is None:
+        count, idx = empty_mask(H, Nb, dev)
+    if ws is None:
+        ws = torch.empty(workspace_size_host(L, H, Hkv, d, B, S), dtype=torch.uint8, device=dev)
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    if copy_stream is None:
+        if dev not in _copy_streams:
+            _copy_streams[dev] = torch.cuda.Stream(device=dev)
+        copy_stream = _copy_streams[dev]
+    _check(lib().rr_attention_host(qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), L, H, Hkv, d, B, S, float(tau),
+                                   count.data_ptr(), idx.data_ptr(), out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                   s.cuda_stream, copy_stream.cuda_stream), "rr_attention_host")
+    return out, count, idx

@@ -56,6 +56,69 @@ rr_status check_shape(int L, int H, int Hkv, int d, int B, int S, bool need_s) {
   return RR_OK;
 }
 
+// Enqueues the search (pooling or gathers, scores and block mass, Top-tau) with
+// its scratch at ws laid out by w; the caller has validated everything and
+// reset the status word g.status points to.
+rr_status enqueue_search(const void* q, const void* k, int L, int H, int Hkv, int d, int B, int S, float tau,
+                         unsigned flags, int head0, int32_t* count, int32_t* idx, float* mass, uint8_t* ws,
+                         const Layout& w, const rr::DeviceGuardArgs& g, cudaStream_t s) {
+  float* m = mass ? mass : reinterpret_cast<float*>(ws + w.mass);
+  const bool rotate = (flags & RR_VAR_ROTATE) != 0, sampled = (flags & RR_VAR_SAMPLED_KEYS) != 0;
+  const int g_heads = H / Hkv;
+  rr::SearchSources src{q, ws + w.khi, ws + w.klo, 0, 0, head0};
+  if (rotate) {
+    if (rr::launch_gather_rotated(q, ws + w.qs, L, H, H, 1, d, S, s) != cudaSuccess) return RR_ECUDA;
+    src.q = ws + w.qs;
+    src.q_mode = 1;
+  }
+  if (!sampled) {
+    if (rr::launch_pool_keys(k, ws + w.khi, ws + w.klo, L, Hkv, d, S, s) != cudaSuccess) return RR_ECUDA;
+  } else if (rotate) {
+    if (rr::launch_gather_rotated(k, ws + w.ks, L, H, Hkv, g_heads, d, S, s) != cudaSuccess) return RR_ECUDA;
+    src.k_a = src.k_b = ws + w.ks;
+    src.k_mode = 2;
+  } else {
+    src.k_a = src.k_b = k;
+    src.k_mode = 1;
+  }
+  if (rr::launch_search(src, m, L, H, Hkv, d, B, S, g, s) != cudaSuccess) return RR_ECUDA;
+  const int Nb = L / B;
+  if (flags & RR_VAR_GQA_MASK) {
+    float* gm = reinterpret_cast<float*>(ws + w.gmass);
+    if (rr::launch_group_mass(m, gm, Hkv, g_heads, Nb, s) != cudaSuccess) return RR_ECUDA;
+    if (rr::launch_top_tau(gm, Hkv, Nb, tau, count, idx, g_heads, s) != cudaSuccess) return RR_ECUDA;
+  } else {
+    if (rr::launch_top_tau(m, H, Nb, tau, count, idx, 1, s) != cudaSuccess) return RR_ECUDA;
+  }
+  return RR_OK;
+}
+
+// Workspace of rr_attention_host: the status word, two slots of one kv head's
+// device copies (q [L, g, d], k and v [L, 1, d], o [L, g, d]), and the search
+// scratch of one kv head's g heads (its own status word unused).
+struct HostLayout {
+  size_t status, slot[2], q, k, v, o, search, total;
+  Layout sl;
+};
+
+HostLayout carve_host(int L, int H, int Hkv, int d, int B, int S) {
+  HostLayout w;
+  const int g = H / Hkv;
+  const size_t qb = round_up(static_cast<size_t>(L) * g * d * 2), kb = round_up(static_cast<size_t>(L) * d * 2);
+  w.status = 0;
+  w.q = 0;
+  w.k = qb;
+  w.v = qb + kb;
+  w.o = qb + 2 * kb;
+  const size_t slot_bytes = 2 * qb + 2 * kb;
+  w.slot[0] = kAlign;
+  w.slot[1] = kAlign + slot_bytes;
+  w.search = kAlign + 2 * slot_bytes;
+  w.sl = carve(L, g, 1, d, B, S);
+  w.total = w.search + w.sl.total;
+  return w;
+}
+
 rr_status check_ws(void* ws, size_t ws_bytes, const Layout& w) {
   if (!ws) return RR_EINVAL;
   if (reinterpret_cast<uintptr_t>(ws) % kAlign) return RR_EALIGN;
@@ -98,37 +161,9 @@ rr_status rr_search_variant(const void* q, const void* k, int L, int H, int Hkv,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   unsigned int* status = reinterpret_cast<unsigned int*>(ws + w.status);
-  float* m = mass ? mass : reinterpret_cast<float*>(ws + w.mass);
   const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
-  const bool rotate = (flags & RR_VAR_ROTATE) != 0, sampled = (flags & RR_VAR_SAMPLED_KEYS) != 0;
-  const int g_heads = H / Hkv;
   if (cudaMemsetAsync(status, 0, sizeof(unsigned int), s) != cudaSuccess) return RR_ECUDA;
-  rr::SearchSources src{q, ws + w.khi, ws + w.klo, 0, 0};
-  if (rotate) {
-    if (rr::launch_gather_rotated(q, ws + w.qs, L, H, H, 1, d, S, s) != cudaSuccess) return RR_ECUDA;
-    src.q = ws + w.qs;
-    src.q_mode = 1;
-  }
-  if (!sampled) {
-    if (rr::launch_pool_keys(k, ws + w.khi, ws + w.klo, L, Hkv, d, S, s) != cudaSuccess) return RR_ECUDA;
-  } else if (rotate) {
-    if (rr::launch_gather_rotated(k, ws + w.ks, L, H, Hkv, g_heads, d, S, s) != cudaSuccess) return RR_ECUDA;
-    src.k_a = src.k_b = ws + w.ks;
-    src.k_mode = 2;
-  } else {
-    src.k_a = src.k_b = k;
-    src.k_mode = 1;
-  }
-  if (rr::launch_search(src, m, L, H, Hkv, d, B, S, g, s) != cudaSuccess) return RR_ECUDA;
-  const int Nb = L / B;
-  if (flags & RR_VAR_GQA_MASK) {
-    float* gm = reinterpret_cast<float*>(ws + w.gmass);
-    if (rr::launch_group_mass(m, gm, Hkv, g_heads, Nb, s) != cudaSuccess) return RR_ECUDA;
-    if (rr::launch_top_tau(gm, Hkv, Nb, tau, count, idx, g_heads, s) != cudaSuccess) return RR_ECUDA;
-  } else {
-    if (rr::launch_top_tau(m, H, Nb, tau, count, idx, 1, s) != cudaSuccess) return RR_ECUDA;
-  }
-  return RR_OK;
+  return enqueue_search(q, k, L, H, Hkv, d, B, S, tau, flags, 0, count, idx, mass, ws, w, g, s);
 }
 
 rr_status rr_search(const void* q, const void* k, int L, int H, int Hkv, int d, int B, int S, float tau,
@@ -181,6 +216,81 @@ rr_status rr_mask_recall(const float* mass, const int32_t* count, const int32_t*
   if (rr::launch_mask_recall(mass, count, idx, H, Nb, recall, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return RR_ECUDA;
   return RR_OK;
+}
+
+rr_status rr_workspace_size_host(int L, int H, int Hkv, int d, int B, int S, size_t* bytes) {
+  if (!bytes) return RR_EINVAL;
+  rr_status st = check_shape(L, H, Hkv, d, B, S, true);
+  if (st != RR_OK) return st;
+  *bytes = carve_host(L, H, Hkv, d, B, S).total;
+  return RR_OK;
+}
+
+rr_status rr_attention_host(const void* q_host, const void* k_host, const void* v_host, int L, int H, int Hkv,
+                            int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o_host,
+                            void* workspace, size_t workspace_bytes, void* stream, void* copy_stream) {
+  rr_status st = check_shape(L, H, Hkv, d, B, S, true);
+  if (st != RR_OK) return st;
+  if (!(tau > 0.0f) || tau != tau) return RR_EINVAL;
+  if (!q_host || !k_host || !v_host || !o_host || !count || !idx || !workspace) return RR_EINVAL;
+  if (!aligned16(count) || !aligned16(idx)) return RR_EALIGN;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return RR_EALIGN;
+  const HostLayout hl = carve_host(L, H, Hkv, d, B, S);
+  if (workspace_bytes < hl.total) return RR_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t cs = static_cast<cudaStream_t>(copy_stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned int* status = reinterpret_cast<unsigned int*>(ws + hl.status);
+  const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
+  const int gq = H / Hkv, Nb = L / B;
+  const size_t row_q = static_cast<size_t>(H) * d * 2, row_kv = static_cast<size_t>(Hkv) * d * 2;
+  const size_t wq = static_cast<size_t>(gq) * d * 2, wkv = static_cast<size_t>(d) * 2;
+
+  // events: start (prior work on `stream` before the first copy), in[slot]
+  // (copies of a kv head landed), out[slot] (its kernels done), end (last copy)
+  cudaEvent_t ev[6] = {};
+  for (int i = 0; i < 6; ++i) {
+    if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+      return RR_ECUDA;
+    }
+  }
+  cudaEvent_t ev_start = ev[0], ev_end = ev[5];
+  cudaEvent_t ev_in[2] = {ev[1], ev[2]}, ev_out[2] = {ev[3], ev[4]};
+  auto h2d = [&](int c) {
+    uint8_t* base = ws + hl.slot[c & 1];
+    const uint8_t* qh = static_cast<const uint8_t*>(q_host) + c * wq;
+    const uint8_t* kh = static_cast<const uint8_t*>(k_host) + c * wkv;
+    const uint8_t* vh = static_cast<const uint8_t*>(v_host) + c * wkv;
+    return cudaMemcpy2DAsync(base + hl.q, wq, qh, row_q, wq, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+           cudaMemcpy2DAsync(base + hl.k, wkv, kh, row_kv, wkv, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+           cudaMemcpy2DAsync(base + hl.v, wkv, vh, row_kv, wkv, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+           cudaEventRecord(ev_in[c & 1], cs) == cudaSuccess;
+  };
+  bool ok = cudaMemsetAsync(status, 0, sizeof(unsigned int), s) == cudaSuccess &&
+            cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(cs, ev_start, 0) == cudaSuccess;
+  for (int c = 0; c < 2 && c < Hkv && ok; ++c) ok = h2d(c);
+  for (int c = 0; c < Hkv && ok; ++c) {
+    const int slot = c & 1;
+    uint8_t* base = ws + hl.slot[slot];
+    int32_t* cc = count + static_cast<size_t>(c) * gq * Nb;
+    int32_t* ic = idx + static_cast<size_t>(c) * gq * Nb * Nb;
+    ok = cudaStreamWaitEvent(s, ev_in[slot], 0) == cudaSuccess;
+    if (ok) {
+      ok = enqueue_search(base + hl.q, base + hl.k, L, gq, 1, d, B, S, tau, 0u, c * gq, cc, ic, nullptr,
+                          ws + hl.search, hl.sl, g, s) == RR_OK;
+    }
+    ok = ok && rr::launch_bsfa(base + hl.q, base + hl.k, base + hl.v, cc, ic, base + hl.o, L, gq, 1, d, B, g, s) ==
+                   cudaSuccess;
+    ok = ok && cudaEventRecord(ev_out[slot], s) == cudaSuccess && cudaStreamWaitEvent(cs, ev_out[slot], 0) == cudaSuccess;
+    ok = ok && cudaMemcpy2DAsync(static_cast<uint8_t*>(o_host) + c * wq, row_q, base + hl.o, wq, wq, L,
+                                 cudaMemcpyDeviceToHost, cs) == cudaSuccess;
+    // the slot's inputs are free once its kernels are done (waited above)
+    if (ok && c + 2 < Hkv) ok = h2d(c + 2);
+  }
+  ok = ok && cudaEventRecord(ev_end, cs) == cudaSuccess && cudaStreamWaitEvent(s, ev_end, 0) == cudaSuccess;
+  for (int i = 0; i < 6; ++i) cudaEventDestroy(ev[i]);   // released once their work completes
+  return ok ? RR_OK : RR_ECUDA;
 }
 
 rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int Nb, uint8_t* dense, void* stream) {

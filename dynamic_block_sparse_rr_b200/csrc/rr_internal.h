@@ -23,12 +23,15 @@ cudaError_t launch_pool_keys(const void* k, void* khi, void* klo, int L, int Hkv
 //   k_mode 0: k_a / k_b are the stride means' bf16 (hi, lo) parts [Ns, Hkv, d];
 //          1: k_a is k [L, Hkv, d], one key per stride at offset h mod S;
 //          2: k_a holds the sampled keys, gathered into [Ns, H, d].
+// head0: global index of head 0 of this launch (the sampled offsets of q_mode 0
+// and k_mode 1 are (h + head0) mod S), for searches run on a slice of the heads.
 struct SearchSources {
   const void* q;
   const void* k_a;
   const void* k_b;
   int q_mode;
   int k_mode;
+  int head0;
 };
 cudaError_t launch_search(const SearchSources& src, float* mass, int L, int H, int Hkv, int d, int B, int S,
                           const DeviceGuardArgs& g, cudaStream_t stream);

@@ -61,7 +61,7 @@ template <int D, int LOGR>
 __global__ void __launch_bounds__(kThreads, 2)
     search_kernel(const __grid_constant__ CUtensorMap mqs, const __grid_constant__ CUtensorMap mkh,
                   const __grid_constant__ CUtensorMap mkl, float* __restrict__ mass, int H, int Hkv, int S,
-                  int Ns, int Nb, float sl2, int q_mode, int k_mode, unsigned int* status, uint64_t limit_ns) {
+                  int Ns, int Nb, float sl2, int q_mode, int k_mode, int head0, unsigned int* status, uint64_t limit_ns) {
   using C = SearchCfg<D>;
   constexpr int R = 1 << LOGR;                 // sampled rows (and strides) per block
   constexpr int GPT = kTile / R;               // key blocks per 128-stride tile
@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_expect_tx(qb, C::kTileBytes);
       for (int a = 0; a < D / 64; ++a) {
         if (q_mode == 0)
-          tma_load_4d(smem_u32(sQ + a * kTile * 128), &mqs, qb, a * 64, h, h % S, rt * kTile);
+          tma_load_4d(smem_u32(sQ + a * kTile * 128), &mqs, qb, a * 64, h, (h + head0) % S, rt * kTile);
         else
           tma_load_3d(smem_u32(sQ + a * kTile * 128), &mqs, qb, a * 64, h, rt * kTile);
       }
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (k_mode == 0)
               tma_load_3d(da, part == 0 ? &mkh : &mkl, fb, a * 64, kvh, c * kTile);
             else if (k_mode == 1)
-              tma_load_4d(da, &mkh, fb, a * 64, kvh, h % S, c * kTile);
+              tma_load_4d(da, &mkh, fb, a * 64, kvh, (h + head0) % S, c * kTile);
             else
               tma_load_3d(da, &mkh, fb, a * 64, h, c * kTile);
           }
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 template <int D, int LOGR>
 cudaError_t launch_search_t(const CUtensorMap& mqs, const CUtensorMap& mkh, const CUtensorMap& mkl, float* mass,
                             int H, int Hkv, int S, int Ns, int Nb, float sl2, int q_mode, int k_mode,
-                            const DeviceGuardArgs& g, cudaStream_t stream) {
+                            int head0, const DeviceGuardArgs& g, cudaStream_t stream) {
   using C = SearchCfg<D>;
   static bool attr = false;
   if (!attr) {
@@ -298,23 +298,23 @@ cudaError_t launch_search_t(const CUtensorMap& mqs, const CUtensorMap& mkh, cons
   }
   const int n_row_tiles = (Ns + kTile - 1) / kTile;
   search_kernel<D, LOGR><<<static_cast<unsigned>(n_row_tiles) * H, kThreads, C::kSmem, stream>>>(
-      mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, q_mode, k_mode, g.status, g.limit_ns);
+      mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, q_mode, k_mode, head0, g.status, g.limit_ns);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t dispatch_r(int logr, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, float* mass,
-                       int H, int Hkv, int S, int Ns, int Nb, float sl2, int qm, int km, const DeviceGuardArgs& g,
+                       int H, int Hkv, int S, int Ns, int Nb, float sl2, int qm, int km, int h0, const DeviceGuardArgs& g,
                        cudaStream_t st) {
   switch (logr) {
-    case 0: return launch_search_t<D, 0>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
-    case 1: return launch_search_t<D, 1>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
-    case 2: return launch_search_t<D, 2>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
-    case 3: return launch_search_t<D, 3>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
-    case 4: return launch_search_t<D, 4>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
-    case 5: return launch_search_t<D, 5>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
-    case 6: return launch_search_t<D, 6>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
-    case 7: return launch_search_t<D, 7>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, g, st);
+    case 0: return launch_search_t<D, 0>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, h0, g, st);
+    case 1: return launch_search_t<D, 1>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, h0, g, st);
+    case 2: return launch_search_t<D, 2>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, h0, g, st);
+    case 3: return launch_search_t<D, 3>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, h0, g, st);
+    case 4: return launch_search_t<D, 4>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, h0, g, st);
+    case 5: return launch_search_t<D, 5>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, h0, g, st);
+    case 6: return launch_search_t<D, 6>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, h0, g, st);
+    case 7: return launch_search_t<D, 7>(a, b, c, mass, H, Hkv, S, Ns, Nb, sl2, qm, km, h0, g, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -341,8 +341,8 @@ cudaError_t launch_search(const SearchSources& src, float* mass, int L, int H, i
   if (!ok) return cudaErrorInvalidValue;
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
   if (d == 128)
-    return dispatch_r<128>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, src.q_mode, src.k_mode, g, stream);
-  return dispatch_r<64>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, src.q_mode, src.k_mode, g, stream);
+    return dispatch_r<128>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, src.q_mode, src.k_mode, src.head0, g, stream);
+  return dispatch_r<64>(logr, mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, src.q_mode, src.k_mode, src.head0, g, stream);
 }
 
 }  // namespace rr

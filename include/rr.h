@@ -121,6 +121,28 @@ rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H
                        int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/* rr_attention on host-resident tensors, with the host<->device copies
+ * pipelined against the kernels kv head by kv head: the copies of kv head c+2
+ * in and of kv head c out run on `copy_stream` while the search and attention
+ * of kv head c+1 run on `stream`.  Results are those of rr_attention bit for
+ * bit (each kv head's g query heads are searched with their global head index).
+ * In:  q_host [L,H,d], k_host, v_host [L,Hkv,d] bf16, HOST memory (page-locked
+ *      for the copies to be asynchronous; pageable memory works but serialises).
+ * Out: o_host [L,H,d] bf16 host memory; count [H,Nb], idx [H,Nb,Nb] int32
+ *      DEVICE memory.  All caller-owned.
+ * Workspace: rr_workspace_size_host bytes of device memory, 256-byte aligned
+ * (two slots of one kv head's q, k, v, o, and one kv head's search scratch).
+ * Streams: `stream` and `copy_stream` are cudaStream_t; the copy stream first
+ * waits for the work already queued on `stream`, and `stream` finally waits for
+ * the last copy, so synchronising `stream` covers the whole call (o_host is
+ * complete then).  Six CUDA events are created and released per call; no
+ * device memory is allocated.  Validation as rr_attention. */
+rr_status rr_workspace_size_host(int L, int H, int Hkv, int d, int B, int S, size_t* bytes);
+rr_status rr_attention_host(const void* q_host, const void* k_host, const void* v_host, int L, int H,
+                            int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx,
+                            void* o_host, void* workspace, size_t workspace_bytes, void* stream,
+                            void* copy_stream);
+
 /* Mask diagnostics (the synthetic counterpart of the pattern visualisations,
  * Figures 4 and 5: full-attention ground truth against the RR selection).
  * recall[h*Nb+I] = sum of mass[h,I,J] over the J listed in (count, idx) for row

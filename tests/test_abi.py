@@ -160,3 +160,26 @@ def test_search_variant_rejects_before_any_launch(rr):
     assert call(tau=0.0) == rr.RR_EINVAL
     assert call(nws=n - 1) == rr.RR_EINVAL           # the variant workspace is larger than the plain one
     assert n > _ws(L, H, Hkv, d, B, S)[1]
+
+
+def test_host_workspace_and_rejections(rr):
+    lib = rr.lib()
+    g = 1 << 20
+    L, H, Hkv, d, B, S = 4096, 8, 2, 128, 128, 16
+    n = ctypes.c_size_t()
+    assert lib.rr_workspace_size_host(L, H, Hkv, d, B, S, ctypes.byref(n)) == rr.RR_OK
+    gq = H // Hkv
+    # two slots of one kv head's q, k, v, o plus one kv head's search scratch
+    assert n.value >= 2 * (2 * L * gq * d * 2 + 2 * L * d * 2) + gq * (L // B) ** 2 * 4
+    assert lib.rr_workspace_size_host(L, H, 3, d, B, S, ctypes.byref(n)) == rr.RR_EINVAL
+    nws = rr.workspace_size_host(L, H, Hkv, d, B, S)
+
+    def call(qh=g, oh=g, count=g, ws=g, nb=nws, tau=0.9):
+        return lib.rr_attention_host(qh, g, g, L, H, Hkv, d, B, S, tau, count, g, oh, ws, nb, None, None)
+
+    assert call(qh=None) == rr.RR_EINVAL
+    assert call(oh=None) == rr.RR_EINVAL
+    assert call(count=g + 4) == rr.RR_EALIGN
+    assert call(ws=g + 64) == rr.RR_EALIGN
+    assert call(nb=nws - 1) == rr.RR_EINVAL
+    assert call(tau=0.0) == rr.RR_EINVAL

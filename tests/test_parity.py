@@ -306,3 +306,25 @@ def test_mask_to_dense_matches_lists(rr):
             i2[h, I, :len(sel)] = sel
     dense2 = rr.mask_to_dense(torch.from_numpy(c2).cuda(), torch.from_numpy(i2).cuda()).cpu().numpy()
     assert np.array_equal(dense2.astype(bool), dense_from_lists(c2, i2))
+
+
+@pytest.mark.parametrize("L,H,Hkv,d,B,S,tau,structure", [
+    (2048, 8, 2, 128, 128, 16, 0.9, gen.PLANTED),   # two kv heads: both slots, no reuse
+    (1600, 6, 3, 64, 64, 4, 0.9, gen.PLANTED),      # three kv heads: slot 0 reused, ragged tile
+    (4096, 7, 1, 128, 128, 16, 0.95, gen.VIDEO),    # one kv head: a single chunk
+    (2048, 16, 8, 128, 64, 8, 0.8, gen.IID),        # eight kv heads, B = 64
+])
+def test_attention_host_matches_device_path(rr, L, H, Hkv, d, B, S, tau, structure):
+    """rr_attention_host (host buffers, copies pipelined per kv head) returns the
+    device path's output and mask bit for bit."""
+    q, k, v = gen.make_qkv(L, H, Hkv, d, structure, 31)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    o_d, c_d, i_d = rr.attention(qd, kd, vd, B, S, tau)
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    o_h, c_h, i_h = rr.attention_host(pin(q), pin(k), pin(v), B, S, tau)
+    torch.cuda.synchronize()
+    assert torch.equal(c_h, c_d)
+    Nb = L // B
+    cols = torch.arange(Nb, device="cuda")[None, None, :] < c_d[:, :, None]
+    assert torch.equal(torch.where(cols, i_h, 0), torch.where(cols, i_d, 0))
+    assert torch.equal(o_h.view(torch.int16), o_d.cpu().view(torch.int16))
