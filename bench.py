@@ -203,7 +203,7 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -421,6 +421,60 @@ def run_recall(args, cfg, taus, variants=(0,)):
                       "config": workload_config(cfg, taus[0]), "rows": rows, "search_ms": search_ms}), flush=True)
 
 
+def run_sweep(args):
+    """Per-config table (diagnostic, not the contract line): for every config
+    and tau, search and attention ms (mean of `steps` after `warmup`), attention
+    TFLOP/s over visited blocks and its share of the measured sustained peak,
+    the visited fraction, and the speedup over the same kernel on every causal
+    block.  One JSON line per (config, tau)."""
+    import torch
+    import dynamic_block_sparse_rr_b200 as rr
+    dev = torch.device("cuda", 0)
+    peaks = measured_peaks()
+    peak = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
+    for name in ("llama16k", "llama32k", "video64k", "llama128k"):
+        cfg = gen.CONFIGS[name]
+        q, k, v = gen.make_config(cfg)
+        to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+        del q, k, v
+        L, H, Hkv, d, B, S = cfg.L, cfg.H, cfg.Hkv, cfg.d, cfg.B, cfg.S
+        Nb = L // B
+        ws = rr.workspace(L, H, Hkv, d, B, S, dev)
+        count, idx = rr.empty_mask(H, Nb, dev)
+        o = torch.empty_like(qd)
+        stream = torch.cuda.current_stream(dev)
+
+        def timed(fn, reps):
+            for _ in range(args.warmup):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            return e0.elapsed_time(e1) / reps
+
+        cd, idd = rr.empty_mask(H, Nb, dev)
+        rr.search(qd, kd, B, S, 1.0, count=cd, idx=idd, ws=ws)
+        dense_ms = timed(lambda: rr.sparse_attn(qd, kd, vd, cd, idd, B, out=o, ws=ws), args.steps)
+        for tau in cfg.taus:
+            search_ms = timed(lambda: rr.search(qd, kd, B, S, tau, count=count, idx=idx, ws=ws), args.steps)
+            attn_ms = timed(lambda: rr.sparse_attn(qd, kd, vd, count, idx, B, out=o, ws=ws), args.steps)
+            if rr.check_status(ws) != rr.RR_OK:
+                raise RuntimeError("device-side status %d" % rr.check_status(ws))
+            visited = int(count.sum().item())
+            tf = block_flops(cfg, visited) / (attn_ms / 1e3) / 1e12
+            print(json.dumps({"sweep": name, "tau": tau, "search_ms": search_ms, "attn_ms": attn_ms,
+                              "step_ms": search_ms + attn_ms, "attn_tflops": tf, "attn_frac_of_sustained": tf / peak,
+                              "visited_fraction": visited / (H * Nb * (Nb + 1) / 2), "dense_attn_ms": dense_ms,
+                              "speedup_vs_dense": dense_ms / (search_ms + attn_ms),
+                              "search_share": search_ms / (search_ms + attn_ms)}), flush=True)
+        del qd, kd, vd, ws, count, idx, o, cd, idd
+        torch.cuda.empty_cache()
+
+
 def variant_name(flags: int) -> str:
     """rr: the plain search; rot / sk / gqa: the sampling variants of rr_search_variant."""
     parts = [n for bit, n in ((1, "rot"), (2, "sk"), (4, "gqa")) if flags & bit]
@@ -441,6 +495,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--recall", action="store_true",
                     help="mask diagnostics instead of timing: recall of exact attention mass per tau")
+    ap.add_argument("--sweep", action="store_true",
+                    help="per-config table instead of the contract line: every config and tau")
     ap.add_argument("--variants", default="0",
                     help="with --recall: comma-separated sampling-variant flags (1 rotate, 2 sampled keys, "
                          "4 GQA mask; 0 the plain search)")
@@ -457,6 +513,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, cfg, tau, world)
+        return
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args)
         return
     if args.recall:
         if rank == 0:
