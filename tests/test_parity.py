@@ -328,3 +328,24 @@ def test_attention_host_matches_device_path(rr, L, H, Hkv, d, B, S, tau, structu
     cols = torch.arange(Nb, device="cuda")[None, None, :] < c_d[:, :, None]
     assert torch.equal(torch.where(cols, i_h, 0), torch.where(cols, i_d, 0))
     assert torch.equal(o_h.view(torch.int16), o_d.cpu().view(torch.int16))
+
+
+@pytest.mark.slow
+def test_attention_host_llama128k_matches_device_path(rr):
+    """The end-to-end path at the benchmark size (128K, the launch configuration
+    the bench times): rr_attention_host output and mask equal the device path's
+    bit for bit."""
+    cfg = gen.CONFIGS["llama128k"]
+    q, k, v = gen.make_config(cfg)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    o_d, c_d, i_d = rr.attention(qd, kd, vd, cfg.B, cfg.S, cfg.tau)
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    qh, kh, vh = pin(q), pin(k), pin(v)
+    del q, k, v
+    o_h, c_h, i_h = rr.attention_host(qh, kh, vh, cfg.B, cfg.S, cfg.tau)
+    torch.cuda.synchronize()
+    assert torch.equal(c_h, c_d)
+    Nb = cfg.L // cfg.B
+    cols = torch.arange(Nb, device="cuda")[None, None, :] < c_d[:, :, None]
+    assert torch.equal(torch.where(cols, i_h, 0), torch.where(cols, i_d, 0))
+    assert torch.equal(o_h.view(torch.int16), o_d.cpu().view(torch.int16))

@@ -113,3 +113,15 @@ def test_flags_zero_is_rr_search(rr):
     Nb = L // B
     cols = torch.arange(Nb, device="cuda")[None, None, :] < c0[:, :, None]
     assert torch.equal(torch.where(cols, i0, 0), torch.where(cols, i1, 0))
+
+
+@pytest.mark.slow
+def test_sampled_keys_video64k_full_size(rr):
+    """Sampled keys (and the GQA mask on top) on the full video workload
+    (H=28/Hkv=4, L=65536): masks against the oracle's in full."""
+    cfg = gen.CONFIGS["video64k"]
+    for flags in (SK, SK | GQA):
+        count, idx, st = run_case(rr, cfg.L, cfg.H, cfg.Hkv, cfg.d, cfg.B, cfg.S, cfg.tau, flags,
+                                  cfg.structure, seed=cfg.seed)
+        Nb = cfg.L // cfg.B
+        print(flags, st, "visited", count.sum() / (cfg.H * Nb * (Nb + 1) / 2))
