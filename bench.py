@@ -458,10 +458,15 @@ def run_sweep(args):
 
         cd, idd = rr.empty_mask(H, Nb, dev)
         rr.search(qd, kd, B, S, 1.0, count=cd, idx=idd, ws=ws)
-        dense_ms = timed(lambda: rr.sparse_attn(qd, kd, vd, cd, idd, B, out=o, ws=ws), args.steps)
         for tau in cfg.taus:
             search_ms = timed(lambda: rr.search(qd, kd, B, S, tau, count=count, idx=idx, ws=ws), args.steps)
-            attn_ms = timed(lambda: rr.sparse_attn(qd, kd, vd, count, idx, B, out=o, ws=ws), args.steps)
+            # sparse and dense attention alternate, round by round, so that both
+            # see the same clocks (the power-capped clock drifts over a run)
+            a_ms, d_ms = [], []
+            for _ in range(3):
+                a_ms.append(timed(lambda: rr.sparse_attn(qd, kd, vd, count, idx, B, out=o, ws=ws), args.steps))
+                d_ms.append(timed(lambda: rr.sparse_attn(qd, kd, vd, cd, idd, B, out=o, ws=ws), args.steps))
+            attn_ms, dense_ms = statistics.mean(a_ms), statistics.mean(d_ms)
             if rr.check_status(ws) != rr.RR_OK:
                 raise RuntimeError("device-side status %d" % rr.check_status(ws))
             visited = int(count.sum().item())
