@@ -506,13 +506,9 @@ cudaError_t launch_bsfa_t(const CUtensorMap& mq, const CUtensorMap& mk, const CU
                           const int32_t* count, const int32_t* idx, void* o, int H, int Hkv, int Nb, float sl2,
                           const DeviceGuardArgs& g, int inject, cudaStream_t stream) {
   using C = FaCfg<BN, D>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e =
-        cudaFuncSetAttribute(bsfa_kernel<BN, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = set_smem_limit_once(bsfa_kernel<BN, D>, C::kSmem, smem_set);
+  if (e != cudaSuccess) return e;
   bsfa_kernel<BN, D><<<static_cast<unsigned>(H) * Nb, kThreads, C::kSmem, stream>>>(
       mq, mk, mv, count, idx, static_cast<__nv_bfloat16*>(o), H, Hkv, Nb, sl2, g.status, g.limit_ns, inject);
   return cudaGetLastError();

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace rr {
 
 struct DeviceGuardArgs {
@@ -62,6 +64,21 @@ cudaError_t launch_mask_to_dense(const int32_t* count, const int32_t* idx, int H
 // Share of each row's block mass kept by a mask (diagnostics).
 cudaError_t launch_mask_recall(const float* mass, const int32_t* count, const int32_t* idx, int H, int Nb,
                                float* recall, cudaStream_t stream);
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per device
+// (the attribute belongs to the current device's context): `done` holds one
+// bit per device index below 64; higher indices set it on every call.
+template <typename Kernel>
+cudaError_t set_smem_limit_once(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Low byte of the workspace status word when a device-side wait ran out.
 constexpr unsigned kStatusTimeoutCode = 5u;

@@ -289,13 +289,9 @@ cudaError_t launch_search_t(const CUtensorMap& mqs, const CUtensorMap& mkh, cons
                             int H, int Hkv, int S, int Ns, int Nb, float sl2, int q_mode, int k_mode,
                             int head0, const DeviceGuardArgs& g, cudaStream_t stream) {
   using C = SearchCfg<D>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(search_kernel<D, LOGR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = set_smem_limit_once(search_kernel<D, LOGR>, C::kSmem, smem_set);
+  if (e != cudaSuccess) return e;
   const int n_row_tiles = (Ns + kTile - 1) / kTile;
   search_kernel<D, LOGR><<<static_cast<unsigned>(n_row_tiles) * H, kThreads, C::kSmem, stream>>>(
       mqs, mkh, mkl, mass, H, Hkv, S, Ns, Nb, sl2, q_mode, k_mode, head0, g.status, g.limit_ns);

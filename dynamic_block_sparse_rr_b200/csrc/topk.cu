@@ -153,13 +153,9 @@ cudaError_t launch_top_tau(const float* mass, int H, int Nb, float tau, int32_t*
   int p2 = 1;
   while (p2 < Nb) p2 <<= 1;
   const size_t smem = static_cast<size_t>(p2) * 8 + static_cast<size_t>(Nb);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(top_tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(8 * kMaxBlocks + kMaxBlocks));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = set_smem_limit_once(top_tau_kernel, static_cast<int>(8 * kMaxBlocks + kMaxBlocks), smem_set);
+  if (e != cudaSuccess) return e;
   top_tau_kernel<<<static_cast<unsigned>(H) * Nb, kThreads, smem, stream>>>(mass, H, Nb, tau, count, idx, p2, rep);
   return cudaGetLastError();
 }
