@@ -246,24 +246,26 @@ rr_status rr_attention_host(const void* q_host, const void* k_host, const void* 
   const size_t row_q = static_cast<size_t>(H) * d * 2, row_kv = static_cast<size_t>(Hkv) * d * 2;
   const size_t wq = static_cast<size_t>(gq) * d * 2, wkv = static_cast<size_t>(d) * 2;
 
-  // events: start (prior work on `stream` before the first copy), in[slot]
-  // (copies of a kv head landed), out[slot] (its kernels done), end (last copy)
-  cudaEvent_t ev[6] = {};
-  for (int i = 0; i < 6; ++i) {
+  // events: start (prior work on `stream` before the first copy), qk[slot]
+  // (q and k of a kv head landed: its search may start), in[slot] (v landed
+  // too), out[slot] (its kernels done), end (last copy)
+  cudaEvent_t ev[8] = {};
+  for (int i = 0; i < 8; ++i) {
     if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
       for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
       return RR_ECUDA;
     }
   }
   cudaEvent_t ev_start = ev[0], ev_end = ev[5];
-  cudaEvent_t ev_in[2] = {ev[1], ev[2]}, ev_out[2] = {ev[3], ev[4]};
+  cudaEvent_t ev_in[2] = {ev[1], ev[2]}, ev_out[2] = {ev[3], ev[4]}, ev_qk[2] = {ev[6], ev[7]};
   auto h2d = [&](int c) {
     uint8_t* base = ws + hl.slot[c & 1];
     const uint8_t* qh = static_cast<const uint8_t*>(q_host) + c * wq;
     const uint8_t* kh = static_cast<const uint8_t*>(k_host) + c * wkv;
     const uint8_t* vh = static_cast<const uint8_t*>(v_host) + c * wkv;
-    return cudaMemcpy2DAsync(base + hl.q, wq, qh, row_q, wq, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
-           cudaMemcpy2DAsync(base + hl.k, wkv, kh, row_kv, wkv, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+    return cudaMemcpy2DAsync(base + hl.k, wkv, kh, row_kv, wkv, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+           cudaMemcpy2DAsync(base + hl.q, wq, qh, row_q, wq, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+           cudaEventRecord(ev_qk[c & 1], cs) == cudaSuccess &&
            cudaMemcpy2DAsync(base + hl.v, wkv, vh, row_kv, wkv, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
            cudaEventRecord(ev_in[c & 1], cs) == cudaSuccess;
   };
@@ -275,11 +277,12 @@ rr_status rr_attention_host(const void* q_host, const void* k_host, const void* 
     uint8_t* base = ws + hl.slot[slot];
     int32_t* cc = count + static_cast<size_t>(c) * gq * Nb;
     int32_t* ic = idx + static_cast<size_t>(c) * gq * Nb * Nb;
-    ok = cudaStreamWaitEvent(s, ev_in[slot], 0) == cudaSuccess;
+    ok = cudaStreamWaitEvent(s, ev_qk[slot], 0) == cudaSuccess;
     if (ok) {
       ok = enqueue_search(base + hl.q, base + hl.k, L, gq, 1, d, B, S, tau, 0u, c * gq, cc, ic, nullptr,
                           ws + hl.search, hl.sl, g, s) == RR_OK;
     }
+    ok = ok && cudaStreamWaitEvent(s, ev_in[slot], 0) == cudaSuccess;
     ok = ok && rr::launch_bsfa(base + hl.q, base + hl.k, base + hl.v, cc, ic, base + hl.o, L, gq, 1, d, B, g, s) ==
                    cudaSuccess;
     ok = ok && cudaEventRecord(ev_out[slot], s) == cudaSuccess && cudaStreamWaitEvent(cs, ev_out[slot], 0) == cudaSuccess;
@@ -289,7 +292,7 @@ rr_status rr_attention_host(const void* q_host, const void* k_host, const void* 
     if (ok && c + 2 < Hkv) ok = h2d(c + 2);
   }
   ok = ok && cudaEventRecord(ev_end, cs) == cudaSuccess && cudaStreamWaitEvent(s, ev_end, 0) == cudaSuccess;
-  for (int i = 0; i < 6; ++i) cudaEventDestroy(ev[i]);   // released once their work completes
+  for (int i = 0; i < 8; ++i) cudaEventDestroy(ev[i]);   // released once their work completes
   return ok ? RR_OK : RR_ECUDA;
 }
 

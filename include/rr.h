@@ -124,7 +124,8 @@ rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H
 /* rr_attention on host-resident tensors, with the host<->device copies
  * pipelined against the kernels kv head by kv head: the copies of kv head c+2
  * in and of kv head c out run on `copy_stream` while the search and attention
- * of kv head c+1 run on `stream`.  Results are those of rr_attention bit for
+ * of kv head c+1 run on `stream` (a kv head's search starts once its q and k
+ * have landed, its attention once v has too).  Results are those of rr_attention bit for
  * bit (each kv head's g query heads are searched with their global head index).
  * In:  q_host [L,H,d], k_host, v_host [L,Hkv,d] bf16, HOST memory (page-locked
  *      for the copies to be asynchronous; pageable memory works but serialises).
@@ -135,7 +136,7 @@ rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H
  * Streams: `stream` and `copy_stream` are cudaStream_t; the copy stream first
  * waits for the work already queued on `stream`, and `stream` finally waits for
  * the last copy, so synchronising `stream` covers the whole call (o_host is
- * complete then).  Six CUDA events are created and released per call; no
+ * complete then).  Eight CUDA events are created and released per call; no
  * device memory is allocated.  Validation as rr_attention. */
 rr_status rr_workspace_size_host(int L, int H, int Hkv, int d, int B, int S, size_t* bytes);
 rr_status rr_attention_host(const void* q_host, const void* k_host, const void* v_host, int L, int H,
