@@ -437,12 +437,14 @@ def run_sweep(args):
     and tau, search and attention ms (mean of `steps` after `warmup`), attention
     TFLOP/s over visited blocks and its share of the measured sustained peak,
     the visited fraction, and the speedup over the same kernel on every causal
-    block.  One JSON line per (config, tau)."""
+    block.  One JSON line per (config, tau, sampling variant); `--variants`
+    picks the variants (0: the plain search)."""
     import torch
     import dynamic_block_sparse_rr_b200 as rr
     dev = torch.device("cuda", 0)
     peaks = measured_peaks()
     peak = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
+    variants = [int(f) for f in args.variants.split(",")]
     for name in ("llama16k", "llama32k", "video64k", "llama128k"):
         cfg = gen.CONFIGS[name]
         q, k, v = gen.make_config(cfg)
@@ -451,7 +453,9 @@ def run_sweep(args):
         del q, k, v
         L, H, Hkv, d, B, S = cfg.L, cfg.H, cfg.Hkv, cfg.d, cfg.B, cfg.S
         Nb = L // B
-        ws = rr.workspace(L, H, Hkv, d, B, S, dev)
+        # room for every variant asked for and for the plain search (the sizes differ either way)
+        ws_bytes = max(rr.workspace_size_variant(L, H, Hkv, d, B, S, f) for f in set(variants) | {0})
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         count, idx = rr.empty_mask(H, Nb, dev)
         o = torch.empty_like(qd)
         stream = torch.cuda.current_stream(dev)
@@ -469,8 +473,8 @@ def run_sweep(args):
 
         cd, idd = rr.empty_mask(H, Nb, dev)
         rr.search(qd, kd, B, S, 1.0, count=cd, idx=idd, ws=ws)
-        for tau in cfg.taus:
-            search_ms = timed(lambda: rr.search(qd, kd, B, S, tau, count=count, idx=idx, ws=ws), args.steps)
+        for tau, flags in [(t, f) for t in cfg.taus for f in variants]:
+            search_ms = timed(lambda: rr.search_variant(qd, kd, B, S, tau, flags, count, idx, ws=ws), args.steps)
             # sparse and dense attention alternate, round by round, so that both
             # see the same clocks (the power-capped clock drifts over a run)
             a_ms, d_ms = [], []
@@ -482,7 +486,7 @@ def run_sweep(args):
                 raise RuntimeError("device-side status %d" % rr.check_status(ws))
             visited = int(count.sum().item())
             tf = block_flops(cfg, visited) / (attn_ms / 1e3) / 1e12
-            print(json.dumps({"sweep": name, "tau": tau, "search_ms": search_ms, "attn_ms": attn_ms,
+            print(json.dumps({"sweep": name, "tau": tau, "variant": variant_name(flags), "search_ms": search_ms, "attn_ms": attn_ms,
                               "step_ms": search_ms + attn_ms, "attn_tflops": tf, "attn_frac_of_sustained": tf / peak,
                               "visited_fraction": visited / (H * Nb * (Nb + 1) / 2), "dense_attn_ms": dense_ms,
                               "speedup_vs_dense": dense_ms / (search_ms + attn_ms),
@@ -514,8 +518,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="per-config table instead of the contract line: every config and tau")
     ap.add_argument("--variants", default="0",
-                    help="with --recall: comma-separated sampling-variant flags (1 rotate, 2 sampled keys, "
-                         "4 GQA mask; 0 the plain search)")
+                    help="with --recall or --sweep: comma-separated sampling-variant flags (1 rotate, "
+                         "2 sampled keys, 4 GQA mask; 0 the plain search)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("note: fewer than 3 warm-up steps requested", file=sys.stderr)
