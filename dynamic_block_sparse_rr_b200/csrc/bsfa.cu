@@ -16,10 +16,12 @@
 // exactly in the epilogue:  O = (O_a 2^(m_a-m) + O_b 2^(m_b-m)) / (l_a 2^(m_a-m)
 // + l_b 2^(m_b-m)).
 //
-// Online softmax in the exp2 domain with a lazy rescale: the running max is
-// only moved (and O rescaled in TMEM) when a row's new max exceeds it by more
-// than 8 (a factor 256), which keeps P <= 256 and is exact after the final
-// division because P and l always use the same max.
+// Online softmax in the exp2 domain with a lazy running max: a group's first
+// block sets it to that block's row max; later blocks are exponentiated with
+// it directly, and a row's max moves (with O and l rescaled) only when the
+// block's sum of P passes 2^16.  That keeps P < 2^16, which bf16 and fp32 hold
+// without loss, and is exact after the final division because P and l always
+// use the same max.
 //
 // Warp roles (384 threads, three warpgroups): warp 0 TMA producer; warps 1 and
 // 3 MMA issuers (one thread each) for softmax groups 0 and 1, taking strict
@@ -29,7 +31,8 @@
 // gives registers back (setmaxnreg 48) so that the softmax groups can hold a
 // full 128-column score row (setmaxnreg 224): 128*48 + 256*224 <= 384*168.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512);
-// P_x overwrites the first B/2 columns of S_x.
+// P_x overwrites the last B/2 columns of S_x, so that the first half of the
+// scores is still there when a row's block has to be redone.
 // K/V tiles stream through a 4-stage shared-memory ring in the order the MMA
 // consumes them: K0, K1, V0, K2, V1, K3, ...
 #include <cuda_bf16.h>
@@ -49,13 +52,6 @@ constexpr int kStages = 4;
 // (ex2_fma_x2) instead of MUFU; 0 keeps every exp2 on MUFU.
 #ifndef RR_EMU_EVERY
 #define RR_EMU_EVERY 0
-#endif
-
-// 1: after a group's first block, exponentiate with the running max while the
-// block max is found alongside (rows whose max jumps are redone); 0 (default,
-// measured faster): max first.
-#ifndef RR_SPEC_MAX
-#define RR_SPEC_MAX 0
 #endif
 
 template <int BN, int D>
@@ -89,28 +85,20 @@ struct FaCtrl {
 
 // Exponentiate one row of scores into P = 2^(s*sl2 - m) (bf16, written to TMEM
 // at p_col) and return the row sum of P in fp32.  kEmu > 0 moves every kEmu-th
-// pair from MUFU to the FMA pipe (ex2_fma_x2); kMax also returns the row max of
-// s, computed on the ALU alongside the exponentials.
-template <int BN, int kEmu, bool kMax>
-__device__ __forceinline__ float exp_store(const float (&s)[BN], float sl2, float m_run, uint32_t p_col,
-                                           float& mx_out) {
+// pair from MUFU to the FMA pipe (ex2_fma_x2).
+template <int BN, int kEmu>
+__device__ __forceinline__ float exp_store(const float (&s)[BN], float sl2, float m_run, uint32_t p_col) {
   const uint64_t scale2 = f2pack(sl2, sl2);
   const uint64_t negm2 = f2pack(-m_run, -m_run);
   uint64_t acc[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) acc[j] = 0ull;   // (+0.0f, +0.0f)
-  float m8[8];
-  if constexpr (kMax) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) m8[j] = -INFINITY;
-  }
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t pk[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int jj = c * 16 + j;
-      if constexpr (kMax) m8[j & 7] = max3(m8[j & 7], s[2 * jj], s[2 * jj + 1]);
       const uint64_t xp = fma2(f2pack(s[2 * jj], s[2 * jj + 1]), scale2, negm2);
       uint64_t pp;
       if (kEmu > 0 && (jj % (kEmu > 0 ? kEmu : 1)) == kEmu - 1) {
@@ -127,8 +115,6 @@ __device__ __forceinline__ float exp_store(const float (&s)[BN], float sl2, floa
     }
     tmem_st16(p_col + c * 16, pk);
   }
-  if constexpr (kMax)
-    mx_out = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
   const uint64_t t = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
   float lo, hi;
   f2unpack(t, lo, hi);
@@ -158,7 +144,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = FaCfg<BN, D>;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, BN, false, false);
   constexpr uint32_t kIdO = idesc_bf16_f32(128, D, false, true);
-  constexpr float kRescale = 8.0f;
+  // A row's running max moves only when one block's exponentials sum past
+  // this bound, so every P stays below 2^16: bf16 and fp32 share the 8-bit
+  // exponent, and P, O and the row sum lose nothing at that size.
+  constexpr float kSumLimit = 65536.0f;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -299,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vb = v_lo + st * kStageStep;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts_lh(o_tm, s_tm + kk * 8, vb + kk * (16 * 128 >> 4), v_hi, kIdO, (acc || kk > 0) ? 1u : 0u);
+          umma_ts_lh(o_tm, s_tm + BN / 2 + kk * 8, vb + kk * (16 * 128 >> 4), v_hi, kIdO, (acc || kk > 0) ? 1u : 0u);
         umma_commit(smem_u32(&ctl->empty[st]));
       };
       volatile int* turn = &ctl->turn;
@@ -361,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = wq * 32 + lane;             // row of the query tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t s_col = tm + lane_off + x * 128;
+    const uint32_t p_col = s_col + BN / 2;
     const uint32_t o_col = tm + lane_off + 256 + x * 128;
     const int n_a = (cnt + 1) >> 1, n_b = cnt >> 1;
     const int n_x = x == 0 ? n_a : n_b;
@@ -386,47 +376,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < BN; ++j)
           if (j > row) s[j] = -INFINITY;                // causal mask inside block J == I
       }
-      // Online softmax with a lazy rescale: the running max moves (and O is
-      // rescaled in TMEM) only when a row's block max exceeds it by more than 8.
-      // After the first block the exponentials start at once with the running
-      // max, the block max being found alongside them; the rare rows whose max
-      // jumps are then redone.  The first block and the masked diagonal block
-      // take the max first.
-      float sum, dummy;
+      // Online softmax with a lazy running max.  A group's first block sets it
+      // to the block's row max.  Later blocks are exponentiated with it at
+      // once, with no max pass: only when a row's block sum passes kSumLimit
+      // (some score grew far above the running max) does that row take its
+      // exact block max, rescale O and l, and redo the block.
+      auto expo = [&]() {
+        if constexpr (RR_EMU_EVERY == 0) {
+          return exp_store<BN, 0>(s, sl2, m_run, p_col);
+        } else {
+          return diag ? exp_store<BN, 0>(s, sl2, m_run, p_col) : exp_store<BN, RR_EMU_EVERY>(s, sl2, m_run, p_col);
+        }
+      };
       bool rescale = false;
       float alpha = 1.0f;
-      if (u == 0 || diag || !RR_SPEC_MAX) {
-        const float m_blk = row_max<BN>(s) * sl2;
-        if (u == 0) {
-          m_run = m_blk;
-        } else {
-          const bool need = m_blk > m_run + kRescale;
-          rescale = __any_sync(0xffffffffu, need);
-          if (need) {
-            alpha = ex2(m_run - m_blk);
-            l_run *= alpha;
-            m_run = m_blk;
-          }
-        }
-        if (diag) {
-          sum = exp_store<BN, 0, false>(s, sl2, m_run, s_col, dummy);
-        } else {
-          sum = exp_store<BN, RR_EMU_EVERY, false>(s, sl2, m_run, s_col, dummy);
-        }
-      } else {
-        float mx;
-        sum = exp_store<BN, RR_EMU_EVERY, true>(s, sl2, m_run, s_col, mx);
-        const float m_blk = mx * sl2;
-        const bool need = m_blk > m_run + kRescale;
+      if (u == 0) m_run = row_max<BN>(s) * sl2;
+      float sum = expo();
+      if (u > 0) {
+        const bool need = !(sum <= kSumLimit);
         rescale = __any_sync(0xffffffffu, need);
         if (rescale) {
-          if (need) {
-            alpha = ex2(m_run - m_blk);
-            l_run *= alpha;
-            m_run = m_blk;
-          }
           tmem_wait_st();
-          sum = exp_store<BN, RR_EMU_EVERY, false>(s, sl2, m_run, s_col, dummy);
+          // The P stores overwrote the second half of the scores in TMEM; the
+          // first half is reloaded, so those registers need not live across
+          // the first pass.
+          if constexpr (BN == 128) {
+            uint32_t r[64];
+            tmem_ld32x2(s_col, s_col + 32, r);
+#pragma unroll
+            for (int j = 0; j < 64; ++j) s[j] = __uint_as_float(r[j]);
+          } else {
+            uint32_t r[32];
+            tmem_ld32(s_col, r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(r[j]);
+          }
+          if (diag) {
+#pragma unroll
+            for (int j = 0; j < BN / 2; ++j)
+              if (j > row) s[j] = -INFINITY;
+          }
+          if (need) {
+            const float m_new = fmaxf(m_run, row_max<BN>(s) * sl2);
+            alpha = ex2(m_run - m_new);
+            l_run *= alpha;
+            m_run = m_new;
+          }
+          sum = expo();
         }
       }
       // O of this group is quiescent here (its last P V completed before this S
