@@ -330,6 +330,24 @@ def test_attention_host_matches_device_path(rr, L, H, Hkv, d, B, S, tau, structu
     assert torch.equal(o_h.view(torch.int16), o_d.cpu().view(torch.int16))
 
 
+def test_attention_host_pinned_and_pageable_outputs_agree(rr):
+    """rr_attention_host fills a caller's page-locked or pageable output with the
+    device path's O, bit for bit."""
+    L, H, Hkv, d, B, S, tau = 3072, 8, 2, 128, 128, 16, 0.9
+    q, k, v = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 33)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    o_d, _, _ = rr.attention(qd, kd, vd, B, S, tau)
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    qh, kh, vh = pin(q), pin(k), pin(v)
+    out_pinned = torch.full((L, H, d), float("nan"), dtype=torch.bfloat16).pin_memory()
+    out_pageable = torch.full((L, H, d), float("nan"), dtype=torch.bfloat16)
+    for out in (out_pinned, out_pageable):
+        o_h, _, _ = rr.attention_host(qh, kh, vh, B, S, tau, out=out)
+        torch.cuda.synchronize()
+        assert o_h.data_ptr() == out.data_ptr()
+        assert torch.equal(o_h.view(torch.int16), o_d.cpu().view(torch.int16))
+
+
 @pytest.mark.slow
 def test_attention_host_llama128k_matches_device_path(rr):
     """The end-to-end path at the benchmark size (128K, the launch configuration
