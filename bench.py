@@ -331,7 +331,7 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
 
     # end to end through the public API with host buffers: rr_attention_host
     # copies q, k, v in and o out (page-locked host memory) inside the call,
-    # pipelined against the kernels kv head by kv head
+    # pipelined against the kernels item by item
     oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(1, min(args.steps, 2))
     ws_host = torch.empty(rr.workspace_size_host(L, H, Hkv, d, B, S), dtype=torch.uint8, device=dev)
@@ -381,7 +381,8 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
             "visited_blocks": visited, "visited_fraction": visited / (H * Nb * (Nb + 1) / 2),
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms_max,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "path": "rr_attention_host: pinned host q/k/v/o, copies pipelined per kv head"},
+                    "path": "rr_attention_host: pinned host q/k/v/o, copies pipelined per item "
+                            "(a kv head; a single query head for the first and last item)"},
             "gpu_launches": gpu_launches, "clocks": clk, "roofline": roofline, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

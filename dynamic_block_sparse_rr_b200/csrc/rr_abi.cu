@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "rr.h"
 #include "rr_internal.h"
 
@@ -244,7 +246,7 @@ rr_status rr_attention_host(const void* q_host, const void* k_host, const void* 
   const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
   const int gq = H / Hkv, Nb = L / B;
   const size_t row_q = static_cast<size_t>(H) * d * 2, row_kv = static_cast<size_t>(Hkv) * d * 2;
-  const size_t wq = static_cast<size_t>(gq) * d * 2, wkv = static_cast<size_t>(d) * 2;
+  const size_t wkv = static_cast<size_t>(d) * 2;
 
   // events: start (prior work on `stream` before the first copy), qk[slot]
   // (q and k of a kv head landed: its search may start), in[slot] (v landed
@@ -258,38 +260,62 @@ rr_status rr_attention_host(const void* q_host, const void* k_host, const void* 
   }
   cudaEvent_t ev_start = ev[0], ev_end = ev[5];
   cudaEvent_t ev_in[2] = {ev[1], ev[2]}, ev_out[2] = {ev[3], ev[4]}, ev_qk[2] = {ev[6], ev[7]};
-  auto h2d = [&](int c) {
-    uint8_t* base = ws + hl.slot[c & 1];
-    const uint8_t* qh = static_cast<const uint8_t*>(q_host) + c * wq;
-    const uint8_t* kh = static_cast<const uint8_t*>(k_host) + c * wkv;
-    const uint8_t* vh = static_cast<const uint8_t*>(v_host) + c * wkv;
+  // Work items: (kv head c, query heads h0 .. h0+gn of its group).  A kv head
+  // is one item, except that the first item holds a single query head (its
+  // inputs land sooner, so the kernels start sooner) and so does the last (its
+  // O copy, which trails the last kernel, is smaller).  Each query head's search
+  // and attention are independent of the others', so the results do not depend
+  // on this split.
+  struct Item { int c, h0, gn; };
+  std::vector<Item> items;
+  for (int c = 0; c < Hkv; ++c) {
+    int h0 = 0, rem = gq;
+    if (c == 0 && rem > 1) { items.push_back({c, 0, 1}); h0 = 1; --rem; }
+    if (c == Hkv - 1 && rem > 1) {
+      items.push_back({c, h0, rem - 1});
+      items.push_back({c, h0 + rem - 1, 1});
+    } else {
+      items.push_back({c, h0, rem});
+    }
+  }
+  const int n_items = static_cast<int>(items.size());
+  auto h2d = [&](int n) {
+    const Item& it = items[n];
+    uint8_t* base = ws + hl.slot[n & 1];
+    const size_t w = static_cast<size_t>(it.gn) * d * 2;   // this item's q (and o) row
+    const uint8_t* qh = static_cast<const uint8_t*>(q_host) + (static_cast<size_t>(it.c) * gq + it.h0) * d * 2;
+    const uint8_t* kh = static_cast<const uint8_t*>(k_host) + it.c * wkv;
+    const uint8_t* vh = static_cast<const uint8_t*>(v_host) + it.c * wkv;
     return cudaMemcpy2DAsync(base + hl.k, wkv, kh, row_kv, wkv, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
-           cudaMemcpy2DAsync(base + hl.q, wq, qh, row_q, wq, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
-           cudaEventRecord(ev_qk[c & 1], cs) == cudaSuccess &&
+           cudaMemcpy2DAsync(base + hl.q, w, qh, row_q, w, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+           cudaEventRecord(ev_qk[n & 1], cs) == cudaSuccess &&
            cudaMemcpy2DAsync(base + hl.v, wkv, vh, row_kv, wkv, L, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
-           cudaEventRecord(ev_in[c & 1], cs) == cudaSuccess;
+           cudaEventRecord(ev_in[n & 1], cs) == cudaSuccess;
   };
   bool ok = cudaMemsetAsync(status, 0, sizeof(unsigned int), s) == cudaSuccess &&
             cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(cs, ev_start, 0) == cudaSuccess;
-  for (int c = 0; c < 2 && c < Hkv && ok; ++c) ok = h2d(c);
-  for (int c = 0; c < Hkv && ok; ++c) {
-    const int slot = c & 1;
+  for (int n = 0; n < 2 && n < n_items && ok; ++n) ok = h2d(n);
+  for (int n = 0; n < n_items && ok; ++n) {
+    const Item& it = items[n];
+    const int slot = n & 1;
     uint8_t* base = ws + hl.slot[slot];
-    int32_t* cc = count + static_cast<size_t>(c) * gq * Nb;
-    int32_t* ic = idx + static_cast<size_t>(c) * gq * Nb * Nb;
+    const int h_first = it.c * gq + it.h0;   // global index of the item's first query head
+    const size_t w = static_cast<size_t>(it.gn) * d * 2;
+    int32_t* cc = count + static_cast<size_t>(h_first) * Nb;
+    int32_t* ic = idx + static_cast<size_t>(h_first) * Nb * Nb;
     ok = cudaStreamWaitEvent(s, ev_qk[slot], 0) == cudaSuccess;
     if (ok) {
-      ok = enqueue_search(base + hl.q, base + hl.k, L, gq, 1, d, B, S, tau, 0u, c * gq, cc, ic, nullptr,
+      ok = enqueue_search(base + hl.q, base + hl.k, L, it.gn, 1, d, B, S, tau, 0u, h_first, cc, ic, nullptr,
                           ws + hl.search, hl.sl, g, s) == RR_OK;
     }
     ok = ok && cudaStreamWaitEvent(s, ev_in[slot], 0) == cudaSuccess;
-    ok = ok && rr::launch_bsfa(base + hl.q, base + hl.k, base + hl.v, cc, ic, base + hl.o, L, gq, 1, d, B, g, s) ==
-                   cudaSuccess;
+    ok = ok && rr::launch_bsfa(base + hl.q, base + hl.k, base + hl.v, cc, ic, base + hl.o, L, it.gn, 1, d, B, g,
+                               s) == cudaSuccess;
     ok = ok && cudaEventRecord(ev_out[slot], s) == cudaSuccess && cudaStreamWaitEvent(cs, ev_out[slot], 0) == cudaSuccess;
-    ok = ok && cudaMemcpy2DAsync(static_cast<uint8_t*>(o_host) + c * wq, row_q, base + hl.o, wq, wq, L,
-                                 cudaMemcpyDeviceToHost, cs) == cudaSuccess;
+    ok = ok && cudaMemcpy2DAsync(static_cast<uint8_t*>(o_host) + static_cast<size_t>(h_first) * d * 2, row_q,
+                                 base + hl.o, w, w, L, cudaMemcpyDeviceToHost, cs) == cudaSuccess;
     // the slot's inputs are free once its kernels are done (waited above)
-    if (ok && c + 2 < Hkv) ok = h2d(c + 2);
+    if (ok && n + 2 < n_items) ok = h2d(n + 2);
   }
   ok = ok && cudaEventRecord(ev_end, cs) == cudaSuccess && cudaStreamWaitEvent(s, ev_end, 0) == cudaSuccess;
   for (int i = 0; i < 8; ++i) cudaEventDestroy(ev[i]);   // released once their work completes

@@ -122,10 +122,13 @@ rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* rr_attention on host-resident tensors, with the host<->device copies
- * pipelined against the kernels kv head by kv head: the copies of kv head c+2
- * in and of kv head c out run on `copy_stream` while the search and attention
- * of kv head c+1 run on `stream` (a kv head's search starts once its q and k
- * have landed, its attention once v has too).  Results are those of rr_attention bit for
+ * pipelined against the kernels item by item.  An item is one kv head with
+ * its query heads, except that the first item holds only the first query head
+ * and the last item only the last one (the first kernels start sooner, and
+ * the O copy that trails the last kernel is smaller).  The copies of item n+2
+ * in and of item n out run on `copy_stream` while the search and attention of
+ * item n+1 run on `stream` (an item's search starts once its q and k have
+ * landed, its attention once v has too).  Results are those of rr_attention bit for
  * bit (each kv head's g query heads are searched with their global head index).
  * In:  q_host [L,H,d], k_host, v_host [L,Hkv,d] bf16, HOST memory (page-locked
  *      for the copies to be asynchronous; pageable memory works but serialises).
@@ -133,6 +136,7 @@ rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H
  *      DEVICE memory.  All caller-owned.
  * Workspace: rr_workspace_size_host bytes of device memory, 256-byte aligned
  * (two slots of one kv head's q, k, v, o, and one kv head's search scratch).
+ * Host memory: a small list of the items is allocated per call.
  * Streams: `stream` and `copy_stream` are cudaStream_t; the copy stream first
  * waits for the work already queued on `stream`, and `stream` finally waits for
  * the last copy, so synchronising `stream` covers the whole call (o_host is

@@ -309,10 +309,11 @@ def test_mask_to_dense_matches_lists(rr):
 
 
 @pytest.mark.parametrize("L,H,Hkv,d,B,S,tau,structure", [
-    (2048, 8, 2, 128, 128, 16, 0.9, gen.PLANTED),   # two kv heads: both slots, no reuse
-    (1600, 6, 3, 64, 64, 4, 0.9, gen.PLANTED),      # three kv heads: slot 0 reused, ragged tile
-    (4096, 7, 1, 128, 128, 16, 0.95, gen.VIDEO),    # one kv head: a single chunk
-    (2048, 16, 8, 128, 64, 8, 0.8, gen.IID),        # eight kv heads, B = 64
+    (2048, 8, 2, 128, 128, 16, 0.9, gen.PLANTED),   # items 1+3 and 3+1 heads: both slots reused
+    (1600, 6, 3, 64, 64, 4, 0.9, gen.PLANTED),      # five items of 1-2 heads, ragged tile
+    (4096, 7, 1, 128, 128, 16, 0.95, gen.VIDEO),    # one kv head in three items (1, 5, 1 heads)
+    (2048, 16, 8, 128, 64, 8, 0.8, gen.IID),        # ten items, B = 64
+    (1024, 4, 4, 64, 64, 4, 0.9, gen.IID),          # g = 1: one item per kv head
 ])
 def test_attention_host_matches_device_path(rr, L, H, Hkv, d, B, S, tau, structure):
     """rr_attention_host (host buffers, copies pipelined per kv head) returns the
