@@ -156,6 +156,39 @@ def test_arbitrary_masks(rr, B, d):
     assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
 
 
+@pytest.mark.parametrize("slope", [1.5, -1.5, 6.0])
+def test_running_max_moves(rr, slope):
+    """Scores that rise (or fall) steeply from key block to key block.  With a
+    rising slope a row's running max, set by its first block, is far below the
+    later blocks, so their exponentials pass the rescale bound again and again:
+    the rows take the rescale path (exact block max, O and l rescaled, block
+    redone) several times.  At slope 6 the last blocks score ~138 (log2 units)
+    above the first block's max, past the fp32 range, so without that path the
+    outputs would overflow.  A falling slope never moves it.  Outputs against
+    the fp64 oracle over every causal block."""
+    L, H, Hkv, d, B = 2048, 2, 1, 128, 128
+    Nb = L // B
+    q, k, v = gen.make_qkv(L, H, Hkv, d, gen.IID, 41)
+    qn, kn = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k)
+    c = -2.0 + slope * (np.arange(L) // B) if slope > 0 else 10.0 + slope * (np.arange(L) // B)
+    qf = 0.5 * qn
+    qf[:, :, 0] += 12.0                                  # every query along e_0
+    kf = 0.5 * kn
+    kf[:, :, 0] += c[:, None].astype(np.float32)          # key block J scores ~ c(J)
+    to_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+    qb, kb = to_bf16(qf), to_bf16(kf)
+    Q, K = qb.float().numpy(), kb.float().numpy()
+    V = gen.bf16_bits_to_f32(v)
+    count, idx = oracle.full_causal_mask(H, Nb)
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    o = rr.sparse_attn(qb.cuda(), kb.cuda(), to_dev(v), torch.from_numpy(count).cuda(),
+                       torch.from_numpy(idx).cuda(), B, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+    O_ref = oracle.sparse_attention(Q, K, V, count, idx, B)
+    mx, mean = output_errors(gpu_o_f32(o), O_ref)
+    assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
+
+
 def test_deterministic(rr):
     L, H, Hkv, d, B, S = 4096, 8, 2, 128, 128, 16
     q, k, v = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 5)
