@@ -428,8 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O of this group is quiescent here (its last P V completed before this S
       // was signalled), and the next P V is issued only after p_full.
       if (rescale) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {   // rare: not unrolled, so it holds 32 registers only
           uint32_t ov[32];
           tmem_ld32(o_col + c * 32, ov);
 #pragma unroll
