@@ -2,20 +2,22 @@
 // last query block (RRAttention abstract: "adaptive Top-tau selection"; TL;DR:
 // "Top-tau block selection and a static protection of the last query block").
 //
-// One CTA per (head h, query block I).  The kept set of row I is the shortest
-// prefix, in (mass descending, J ascending) order, of the I+1 block masses
-// whose sum reaches tau * (row total).  Rows of up to 256 blocks are sorted
-// outright (bitonic network on 64-bit keys, fp64 running sum).  Longer rows use
-// that such a prefix is every block with mass above a threshold value T plus
-// the lowest-J blocks with mass exactly T, and find T without sorting: the
-// masses are non-negative floats, whose bit patterns order like their values,
-// and a radix select over those bits (4 passes of 8 bits) walks down to T,
-// each pass histogramming (count, mass sum) per digit of the remaining
-// candidates and taking the digit where the running sum from the top crosses
-// the target.  Those sums are exact integers (each mass scaled to a fixed-point
-// fraction of the row total, 2^31 units), so the selection is deterministic.
-// The selected J are written in ascending order (flag + exclusive scan).  Row
-// Nb-1, and every row when tau >= 1, keeps all J <= I.
+// The kept set of row (h, I) is the shortest prefix, in (mass descending, J
+// ascending) order, of its I+1 block masses whose sum reaches tau * (row
+// total).  That prefix is every block with mass above a threshold value T plus
+// the lowest-J blocks with mass exactly T, so T is found without sorting.  The
+// sums are exact integers: each mass is scaled to a fixed-point fraction of the
+// row total (round(mass / total * 2^31) units, the total in fp64), which makes
+// the selection deterministic; it can differ from an exact real-number cut only
+// for a block within ~2^-31 of the row total from tau.  The masses are
+// non-negative floats, whose bit patterns order like their values:
+//   * rows of up to 1024 blocks: one warp per row, T by bisection over its 31
+//     bits (a candidate is kept while the units of the masses at or above it
+//     still reach the target);
+//   * longer rows: one CTA per row, T by a radix select (4 passes of 8 bits,
+//     each histogramming the units of the remaining candidates per digit).
+// The selected J are written in ascending order.  Row Nb-1, and every row when
+// tau >= 1, keeps all J <= I.
 #include <stdint.h>
 
 #include "rr_internal.h"
@@ -26,6 +28,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kPerThread = (kMaxBlocks + kThreads - 1) / kThreads;   // masses owned by one thread
+constexpr int kWarpRow = 1024;   // rows up to this length: one warp per row
 
 // Exclusive block scan of one value per thread; returns the exclusive prefix,
 // writes the block total to *total.  Deterministic order.
@@ -58,93 +61,17 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T* warp_buf, T* total) {
 }
 
 struct SelectShared {
-  uint32_t hcnt[kWarps][256];   // per-warp histograms of the current pass
-  uint32_t hsum[kWarps][256];
+  uint32_t hsum[kWarps][256];   // per-warp histograms (units per digit) of the current pass
   double dbuf[kWarps];
   uint32_t ubuf[kWarps];
-  uint32_t digit, base_sum, base_cnt;
+  uint32_t digit, base_sum;
 };
 
-// Rows up to this length are sorted outright (a 64-bit bitonic network in
-// shared memory): for them the sort costs less than the radix passes' fixed
-// work.
-constexpr int kSmallRow = 256;
-
-struct SmallShared {
-  unsigned long long keys[kSmallRow];
-  unsigned char sel[kSmallRow];
-  double dbuf[kWarps];
-  int ibuf[kWarps];
-  int cut;
-};
-
-// The shortest prefix of the row in (mass descending, J ascending) order whose
-// fp64 running sum reaches tau * total, for n <= kSmallRow; writes the selected
-// J ascending to the rep output heads.
-__device__ __forceinline__ void select_small(const float* __restrict__ m, int n, float tau, SmallShared& sh,
-                                             int32_t* __restrict__ out, long long ostride, int rep,
-                                             int32_t* __restrict__ count, long long orow, int Nb) {
-  unsigned long long* keys = sh.keys;
-  unsigned char* sel = sh.sel;
-  const int tid = threadIdx.x;
-  int p2 = 1;
-  while (p2 < n) p2 <<= 1;
-  // Key = (mass bits, ~J) complemented, so an ascending sort gives mass
-  // descending, then J ascending; padding sorts last.
-  for (int i = tid; i < p2; i += kThreads) {
-    unsigned long long key = ~0ull;
-    if (i < n) {
-      const unsigned mb = __float_as_uint(m[i]);
-      key = ~((static_cast<unsigned long long>(mb) << 32) | static_cast<unsigned long long>(0xFFFFFFFFu - i));
-    }
-    keys[i] = key;
-  }
-  if (tid == 0) sh.cut = n - 1;
-  __syncthreads();
-  for (int kk = 2; kk <= p2; kk <<= 1) {
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < p2; i += kThreads) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long a = keys[i], b = keys[ixj];
-          const bool up = (i & kk) == 0;
-          if (up ? (a > b) : (a < b)) {
-            keys[i] = b;
-            keys[ixj] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  // Running sum in fp64 in sorted order (one entry per thread), first index
-  // reaching tau * total.
-  const double v = tid < n ? static_cast<double>(__uint_as_float(static_cast<unsigned>(~keys[tid] >> 32))) : 0.0;
-  double total;
-  const double run = block_exclusive_scan<double>(v, sh.dbuf, &total) + v;
-  if (tid < n && run >= static_cast<double>(tau) * total) atomicMin(&sh.cut, tid);
-  for (int t = tid; t < n; t += kThreads) sel[t] = 0;
-  __syncthreads();
-  const int cnt = sh.cut + 1;
-  for (int t = tid; t < cnt; t += kThreads)
-    sel[0xFFFFFFFFu - static_cast<unsigned>(~keys[t] & 0xFFFFFFFFull)] = 1;
-  __syncthreads();
-  // Ascending output: exclusive scan of the flags in J order.
-  const int flag = tid < n ? sel[tid] : 0;
-  int tot;
-  const int pos = block_exclusive_scan<int>(flag, sh.ibuf, &tot);
-  if (flag)
-    for (int r = 0; r < rep; ++r) out[r * ostride + pos] = tid;
-  for (int r = tid; r < rep; r += kThreads) count[orow + static_cast<long long>(r) * Nb] = cnt;
-}
-
-// kLarge: rows I >= kSmallRow (radix select); else rows I < kSmallRow (sort).
-// The launch covers rows I_top, I_top - 1, ..., heavier rows first.
-template <bool kLarge>
-__global__ void __launch_bounds__(kThreads, kLarge ? 4 : 1) top_tau_kernel(const float* __restrict__ mass, int H,
-                                                                          int Nb, float tau, int32_t* __restrict__ count,
-                                                                          int32_t* __restrict__ idx, int rep,
-                                                                          int I_top) {
+// Rows longer than kWarpRow blocks: radix select, one CTA per row.  The launch
+// covers rows I_top, I_top - 1, ..., heavier rows first.
+__global__ void __launch_bounds__(kThreads, 4) top_tau_kernel(const float* __restrict__ mass, int H, int Nb,
+                                                             float tau, int32_t* __restrict__ count,
+                                                             int32_t* __restrict__ idx, int rep, int I_top) {
   const int I = I_top - static_cast<int>(blockIdx.x / H);
   const int h = static_cast<int>(blockIdx.x % H);
   const long long row = static_cast<long long>(h) * Nb + I;
@@ -162,11 +89,7 @@ __global__ void __launch_bounds__(kThreads, kLarge ? 4 : 1) top_tau_kernel(const
     return;
   }
 
-  if constexpr (!kLarge) {
-    __shared__ SmallShared ss;
-    select_small(mass + row * Nb, n, tau, ss, out, ostride, rep, count, orow, Nb);
-    return;
-  } else {
+  {
     __shared__ SelectShared sh;
 
     // This thread's contiguous chunk of the row: masses as bit patterns, and the
@@ -198,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, kLarge ? 4 : 1) top_tau_kernel(const
     uint32_t total_i;
     block_exclusive_scan<uint32_t>(lsum, sh.ubuf, &total_i);
 
-    uint32_t T = 0, sum_gt = 0, cnt_gt = 0, k_eq = 1;
+    uint32_t T = 0, sum_gt = 0, k_eq = 1;
     if (total_i == 0) {
       // no mass at all: the order is J ascending and the first block reaches it
       T = 0xFFFFFFFFu;   // nothing is above T; J = 0 is the one block kept
@@ -206,13 +129,10 @@ __global__ void __launch_bounds__(kThreads, kLarge ? 4 : 1) top_tau_kernel(const
       // target: the smallest integer prefix sum that is >= tau * total
       const uint32_t target = static_cast<uint32_t>(
           fmin(ceil(static_cast<double>(tau) * static_cast<double>(total_i)), static_cast<double>(total_i)));
-      uint32_t prefix = 0, base_sum = 0, base_cnt = 0;
+      uint32_t prefix = 0, base_sum = 0;
       for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
-        for (int b = tid; b < kWarps * 256; b += kThreads) {
-          (&sh.hcnt[0][0])[b] = 0u;
-          (&sh.hsum[0][0])[b] = 0u;
-        }
+        for (int b = tid; b < kWarps * 256; b += kThreads) (&sh.hsum[0][0])[b] = 0u;
         __syncthreads();
         // histogram of the candidates: the masses whose higher digits equal the
         // digits chosen so far
@@ -221,9 +141,7 @@ __global__ void __launch_bounds__(kThreads, kLarge ? 4 : 1) top_tau_kernel(const
           if (c0 + e < c1) {
             const uint32_t k = key[e];
             if (pass == 0 || ((k ^ prefix) >> (shift + 8)) == 0u) {
-              const uint32_t d = (k >> shift) & 255u;
-              atomicAdd(&sh.hcnt[warp][d], 1u);
-              atomicAdd(&sh.hsum[warp][d], units(k));
+              atomicAdd(&sh.hsum[warp][(k >> shift) & 255u], units(k));
             }
           }
         }
@@ -231,56 +149,43 @@ __global__ void __launch_bounds__(kThreads, kLarge ? 4 : 1) top_tau_kernel(const
         if (warp == 0) {
           // lane L holds digits 255-8L .. 248-8L (descending); the digit taken is
           // the one where the running sum from the top reaches the target
-          uint32_t bs[8], bc[8], ls = 0, lc = 0;
+          uint32_t bs[8], ls = 0;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const int b = 255 - 8 * lane - k;
-            uint32_t s = 0, c = 0;
+            uint32_t s = 0;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) {
-              s += sh.hsum[w][b];
-              c += sh.hcnt[w][b];
-            }
+            for (int w = 0; w < kWarps; ++w) s += sh.hsum[w][b];
             bs[k] = s;
-            bc[k] = c;
             ls += s;
-            lc += c;
           }
-          uint32_t is = ls, ic = lc;
+          uint32_t is = ls;
 #pragma unroll
           for (int off = 1; off < 32; off <<= 1) {
             const uint32_t ys = __shfl_up_sync(0xffffffffu, is, off);
-            const uint32_t yc = __shfl_up_sync(0xffffffffu, ic, off);
-            if (lane >= off) {
-              is += ys;
-              ic += yc;
-            }
+            if (lane >= off) is += ys;
           }
           const uint32_t need = target - base_sum;   // >= 1, reached inside these candidates
-          uint32_t run = is - ls, runc = ic - lc;
+          uint32_t run = is - ls;
           if (run < need && need <= is) {            // exactly one lane
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               if (run + bs[k] >= need) {
                 sh.digit = static_cast<uint32_t>(255 - 8 * lane - k);
                 sh.base_sum = base_sum + run;
-                sh.base_cnt = base_cnt + runc;
                 break;
               }
               run += bs[k];
-              runc += bc[k];
             }
           }
         }
         __syncthreads();
         prefix |= sh.digit << shift;
         base_sum = sh.base_sum;
-        base_cnt = sh.base_cnt;
         __syncthreads();
       }
       T = prefix;
       sum_gt = base_sum;
-      cnt_gt = base_cnt;
       // the blocks of mass exactly T all have the same units; the lowest-J k_eq
       // of them complete the prefix
       const uint32_t t_val = units(T);
@@ -319,23 +224,157 @@ __global__ void __launch_bounds__(kThreads, kLarge ? 4 : 1) top_tau_kernel(const
   }
 }
 
+// Rows of up to kWarpRow blocks: one warp per row, with the selection of the
+// radix path (the same fixed-point units, target, threshold T and lowest-J rule
+// for masses equal to T) and T found by bisection over its 31 bits instead of
+// histograms: bit by bit from the top, a candidate is kept when the units of
+// the masses at or above it still reach the target.  Lane l holds elements
+// l, l+32, l+64, ... (kSlots of them, unused slots mass 0 and 0 units), so that
+// (slot, lane) order is J order, and ballots give the ranks among equal masses
+// and the output positions.
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);   // same bits on every lane
+  return v;
+}
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) { return __reduce_add_sync(0xffffffffu, v); }
+
+template <int kSlots>
+__global__ void __launch_bounds__(kThreads) top_tau_warp_kernel(const float* __restrict__ mass, int H, int Nb,
+                                                                float tau, int32_t* __restrict__ count,
+                                                                int32_t* __restrict__ idx, int rep, int I_top,
+                                                                int n_rows) {
+  const int lane = threadIdx.x & 31;
+  const int gw = static_cast<int>(blockIdx.x) * kWarps + static_cast<int>(threadIdx.x >> 5);
+  if (gw >= n_rows * H) return;   // whole warps only
+  const int I = I_top - gw / H;   // heavier rows first
+  const int h = gw % H;
+  const long long row = static_cast<long long>(h) * Nb + I;
+  const int n = I + 1;            // <= 32 * kSlots
+  const long long orow = static_cast<long long>(h) * rep * Nb + I;
+  const long long ostride = static_cast<long long>(Nb) * Nb;
+  int32_t* out = idx + orow * Nb;
+  if (I == Nb - 1 || !(tau < 1.0f)) {  // protected last row, or tau >= 1: every causal block
+    for (int r = 0; r < rep; ++r)
+      for (int t = lane; t < n; t += 32) out[r * ostride + t] = t;
+    for (int r = lane; r < rep; r += 32) count[orow + static_cast<long long>(r) * Nb] = n;
+    return;
+  }
+  const float* m = mass + row * Nb;
+  uint32_t key[kSlots], un[kSlots];
+  double local = 0.0;
+#pragma unroll
+  for (int e = 0; e < kSlots; ++e) {
+    key[e] = 0u;
+    const int i = e * 32 + lane;
+    if (i < n) {
+      const float v = m[i];
+      key[e] = __float_as_uint(v);
+      local += static_cast<double>(v);
+    }
+  }
+  const double total = warp_sum_f64(local);
+  // Fixed point: a mass is round(mass / total * 2^31) units (sum <= 2^31 + n/2).
+  const double scale = total > 0.0 ? 2147483648.0 / total : 0.0;
+  auto units = [&](uint32_t k) { return __double2uint_rn(static_cast<double>(__uint_as_float(k)) * scale); };
+  uint32_t lsum = 0;
+#pragma unroll
+  for (int e = 0; e < kSlots; ++e) {
+    un[e] = e * 32 + lane < n ? units(key[e]) : 0u;
+    lsum += un[e];
+  }
+  const uint32_t total_i = warp_sum_u32(lsum);
+
+  uint32_t T = 0xFFFFFFFFu, k_eq = 1;
+  if (total_i != 0) {
+    const uint32_t target = static_cast<uint32_t>(
+        fmin(ceil(static_cast<double>(tau) * static_cast<double>(total_i)), static_cast<double>(total_i)));
+    // the largest T whose masses at or above it reach the target (a mass
+    // present in the row: the sum only changes at present values); unused
+    // slots (key 0, 0 units) never count, since every candidate is >= 1
+    uint32_t P = 0;
+    for (int b = 30; b >= 0; --b) {
+      const uint32_t cand = P | (1u << b);
+      uint32_t sge = 0;
+#pragma unroll
+      for (int e = 0; e < kSlots; ++e) sge += key[e] >= cand ? un[e] : 0u;
+      if (warp_sum_u32(sge) >= target) P = cand;
+    }
+    T = P;
+    uint32_t sgt = 0;
+#pragma unroll
+    for (int e = 0; e < kSlots; ++e) sgt += key[e] > T ? un[e] : 0u;
+    const uint32_t sum_gt = warp_sum_u32(sgt);
+    const uint32_t t_val = units(T);
+    k_eq = t_val > 0 ? (target - sum_gt + t_val - 1) / t_val : 1u;
+  }
+
+  // flags in J order: above T, or equal to T and among the first k_eq equal
+  // (a row without mass keeps J = 0 alone)
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t eq_seen = 0, pos = 0;
+#pragma unroll
+  for (int e = 0; e < kSlots; ++e) {
+    if (e * 32 < n) {   // uniform across the warp
+      const int i = e * 32 + lane;
+      const bool valid = i < n;
+      const bool eq = valid && (total_i == 0 ? i == 0 : key[e] == T);
+      const bool gt = valid && total_i != 0 && key[e] > T;
+      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+      const bool sel = gt || (eq && eq_seen + __popc(eqm & lt) < k_eq);
+      eq_seen += __popc(eqm);
+      const uint32_t sm = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const uint32_t p = pos + __popc(sm & lt);
+        for (int r = 0; r < rep; ++r) out[r * ostride + p] = i;
+      }
+      pos += __popc(sm);
+    }
+  }
+  for (int r = lane; r < rep; r += 32) count[orow + static_cast<long long>(r) * Nb] = static_cast<int32_t>(pos);
+}
+
+template <int kSlots>
+cudaError_t launch_warp_rows(const float* mass, int H, int Nb, float tau, int32_t* count, int32_t* idx, int rep,
+                             int I_top, int n_rows, cudaStream_t stream) {
+  if (n_rows <= 0) return cudaSuccess;
+  const long long warps = static_cast<long long>(H) * n_rows;
+  top_tau_warp_kernel<kSlots><<<static_cast<unsigned>((warps + kWarps - 1) / kWarps), kThreads, 0, stream>>>(
+      mass, H, Nb, tau, count, idx, rep, I_top, n_rows);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_top_tau(const float* mass, int H, int Nb, float tau, int32_t* count, int32_t* idx, int rep,
                            cudaStream_t stream) {
   if (H <= 0 || Nb <= 0) return cudaSuccess;
   if (Nb > kMaxBlocks) return cudaErrorInvalidValue;
-  // rows I >= kSmallRow by radix select, rows below by sorting: two launches
-  const int n_large = Nb > kSmallRow ? Nb - kSmallRow : 0, n_small = Nb - n_large;
-  if (n_large > 0) {
-    top_tau_kernel<true><<<static_cast<unsigned>(H) * n_large, kThreads, 0, stream>>>(mass, H, Nb, tau, count, idx,
-                                                                                      rep, Nb - 1);
+  // Rows I >= kWarpRow: radix select, one CTA per row.  Shorter rows: one warp
+  // per row, in three launches by length (8, 16 or 32 masses per lane).
+  // Heavier rows first.
+  if (Nb > kWarpRow) {
+    top_tau_kernel<<<static_cast<unsigned>(H) * (Nb - kWarpRow), kThreads, 0, stream>>>(mass, H, Nb, tau, count,
+                                                                                       idx, rep, Nb - 1);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  top_tau_kernel<false><<<static_cast<unsigned>(H) * n_small, kThreads, 0, stream>>>(mass, H, Nb, tau, count, idx,
-                                                                                     rep, n_small - 1);
-  return cudaGetLastError();
+  // rows [lo, hi) of the row range a launch covers
+  auto range = [&](int lo, int hi, int& I_top, int& n_rows) {
+    hi = hi < Nb ? hi : Nb;
+    n_rows = hi > lo ? hi - lo : 0;
+    I_top = hi - 1;
+  };
+  int top, nr;
+  cudaError_t e;
+  range(512, kWarpRow, top, nr);
+  if ((e = launch_warp_rows<32>(mass, H, Nb, tau, count, idx, rep, top, nr, stream)) != cudaSuccess) return e;
+  range(256, 512, top, nr);
+  if ((e = launch_warp_rows<16>(mass, H, Nb, tau, count, idx, rep, top, nr, stream)) != cudaSuccess) return e;
+  range(0, 256, top, nr);
+  if ((e = launch_warp_rows<8>(mass, H, Nb, tau, count, idx, rep, top, nr, stream)) != cudaSuccess) return e;
+  return cudaSuccess;
 }
 
 }  // namespace rr
