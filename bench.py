@@ -297,8 +297,10 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     visited = int(count.sum().item())
     flops = block_flops(cfg, visited)
-    # pool, search, top-tau (two launches once rows pass 256 blocks), attention
-    gpu_launches = (4 + (cfg.L // cfg.B > 256)) * args.steps
+    # pool, search, top-tau (one launch per row-length class: rows up to 256,
+    # 512 and 1024 blocks, and longer), attention
+    nb = cfg.L // cfg.B
+    gpu_launches = (3 + 1 + (nb > 256) + (nb > 512) + (nb > 1024)) * args.steps
 
     # dense baseline: the same attention kernel with every causal block on.  The
     # sparse and dense launches alternate, so that both see the same clocks (the
