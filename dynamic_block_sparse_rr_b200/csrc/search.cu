@@ -208,33 +208,69 @@ __global__ void __launch_bounds__(kThreads, 2)
       tmem_ld128(tm + lane_off + b * kTile, raw);
       tc_fence_before();
       mbar_arrive(smem_u32(&ctl->s_empty[b]));
+      // scores of this tile as loaded (scaled inside the exponentials below:
+      // x = s * sl2 - m in one fused multiply-add, the same in both passes)
       float v[128];
-      const bool diag = (c == rt);
 #pragma unroll
-      for (int j = 0; j < 128; ++j) {
-        const float x = __uint_as_float(raw[j]) * sl2;
-        v[j] = (diag && j > row) ? -INFINITY : x;   // stride-causal: j <= i
+      for (int j = 0; j < 128; ++j) v[j] = __uint_as_float(raw[j]);
+      if (c == rt) {   // the diagonal tile (uniform across the CTA): stride-causal, j <= i
+#pragma unroll
+        for (int j = 0; j < 128; ++j)
+          if (j > row) v[j] = -INFINITY;
       }
+      const uint64_t sl2x2 = f2pack(sl2, sl2);
       if (!pass2) {
-        float mx = v[0];
+        // row max: eight independent three-input chains (sl2 > 0 commutes with max)
+        float m8[8];
 #pragma unroll
-        for (int j = 1; j < 128; ++j) mx = fmaxf(mx, v[j]);
+        for (int a = 0; a < 8; ++a) m8[a] = fmaxf(v[2 * a], v[2 * a + 1]);
+#pragma unroll
+        for (int j = 16; j < 128; j += 16) {
+#pragma unroll
+          for (int a = 0; a < 8; ++a) m8[a] = max3(m8[a], v[j + 2 * a], v[j + 2 * a + 1]);
+        }
+        const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
         const float m_new = fmaxf(m_run, mx);
-        float sum = 0.f;
+        const uint64_t negm = f2pack(-m_new, -m_new);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // four packed partial sums
 #pragma unroll
-        for (int j = 0; j < 128; ++j) sum += ex2(v[j] - m_new);
-        l_run = l_run * ex2(m_run - m_new) + sum;
+        for (int jj = 0; jj < 64; ++jj) {
+          float x0, x1;
+          f2unpack(fma2(f2pack(v[2 * jj], v[2 * jj + 1]), sl2x2, negm), x0, x1);
+          acc[jj & 3] = add2(acc[jj & 3], f2pack(ex2(x0), ex2(x1)));
+        }
+        float s0, s1;
+        f2unpack(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), s0, s1);
+        l_run = l_run * ex2(m_run - m_new) + (s0 + s1);
         m_run = m_new;
         if (n == n_key_tiles - 1) lse = m_run + lg2(l_run);
         continue;
       }
       // pass 2: probabilities, summed over each key block's R strides (in place: v[g])
+      const uint64_t negl = f2pack(-lse, -lse);
+      if constexpr (R == 1) {
 #pragma unroll
-      for (int g = 0; g < GPT; ++g) {
-        float acc = 0.f;
+        for (int jj = 0; jj < 64; ++jj) {
+          float x0, x1;
+          f2unpack(fma2(f2pack(v[2 * jj], v[2 * jj + 1]), sl2x2, negl), x0, x1);
+          v[2 * jj] = ex2(x0);
+          v[2 * jj + 1] = ex2(x1);
+        }
+      } else {
 #pragma unroll
-        for (int t = 0; t < R; ++t) acc += ex2(v[g * R + t] - lse);
-        v[g] = acc;
+        for (int g = 0; g < GPT; ++g) {
+          uint64_t acc = 0ull;
+#pragma unroll
+          for (int t = 0; t < R / 2; ++t) {
+            const int jj = g * (R / 2) + t;
+            float x0, x1;
+            f2unpack(fma2(f2pack(v[2 * jj], v[2 * jj + 1]), sl2x2, negl), x0, x1);
+            acc = add2(acc, f2pack(ex2(x0), ex2(x1)));
+          }
+          float s0, s1;
+          f2unpack(acc, s0, s1);
+          v[g] = s0 + s1;
+        }
       }
       // ... and over the R sampled rows of each query block
       if constexpr (R <= 32) {
