@@ -156,8 +156,9 @@ def test_arbitrary_masks(rr, B, d):
     assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
 
 
+@pytest.mark.parametrize("B,d", [(128, 128), (64, 64)])
 @pytest.mark.parametrize("slope", [1.5, -1.5, 6.0])
-def test_running_max_moves(rr, slope):
+def test_running_max_moves(rr, slope, B, d):
     """Scores that rise (or fall) steeply from key block to key block.  With a
     rising slope a row's running max, set by its first block, is far below the
     later blocks, so their exponentials pass the rescale bound again and again:
@@ -166,13 +167,13 @@ def test_running_max_moves(rr, slope):
     above the first block's max, past the fp32 range, so without that path the
     outputs would overflow.  A falling slope never moves it.  Outputs against
     the fp64 oracle over every causal block."""
-    L, H, Hkv, d, B = 2048, 2, 1, 128, 128
+    L, H, Hkv = 16 * B, 2, 1
     Nb = L // B
     q, k, v = gen.make_qkv(L, H, Hkv, d, gen.IID, 41)
     qn, kn = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k)
     c = -2.0 + slope * (np.arange(L) // B) if slope > 0 else 10.0 + slope * (np.arange(L) // B)
     qf = 0.5 * qn
-    qf[:, :, 0] += 12.0                                  # every query along e_0
+    qf[:, :, 0] += 12.0 * np.sqrt(d / 128.0)             # every query along e_0 (same logits at any d)
     kf = 0.5 * kn
     kf[:, :, 0] += c[:, None].astype(np.float32)          # key block J scores ~ c(J)
     to_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
