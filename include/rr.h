@@ -64,7 +64,11 @@ rr_status rr_workspace_size(int L, int H, int Hkv, int d, int B, int S, size_t* 
  *   Mass:     summed over the r x r (row, stride) pairs of block (I, J).
  *   Top-tau:  per row I < Nb-1, blocks in (mass desc, J asc) order, shortest
  *             prefix whose share of the row's mass is >= tau (tau >= 1: all).
- *             Row Nb-1 keeps all blocks.
+ *             Row Nb-1 keeps all blocks.  Shares are summed in fixed point
+ *             (each mass rounded to a multiple of 2^-31 of the row total, the
+ *             total in fp64), so the selection is deterministic; a block whose
+ *             running share lies within ~2^-31 of tau may fall either side of
+ *             the cut compared with exact arithmetic.
  * In:  q [L,H,d], k [L,Hkv,d] bf16 (device); tau > 0.
  * Out: count [H,Nb], idx [H,Nb,Nb] int32 (device, caller-owned).
  *      mass: NULL, or a device [H,Nb,Nb] fp32 buffer that receives the
