@@ -190,6 +190,43 @@ def test_running_max_moves(rr, slope, B, d):
     assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
 
 
+@pytest.mark.parametrize("L,tau", [(65536, 0.9), (131072, 0.5), (131072, 0.97)])
+def test_tied_masses_keep_lowest_blocks(rr, L, tau):
+    """Keys all zero: every score is 0, so sampled row i spreads 1/(i+1) over its
+    strides and every full block of a row gets the same mass, bit for bit; the
+    diagonal block gets less.  The selection must then be the lowest-J full
+    blocks (ties go to the lower J), plus the diagonal only when the full blocks
+    cannot reach tau.  Nb = 1024 and 2048 run every Top-tau path (one warp per
+    row with 8, 16 and 32 masses per lane, and one CTA per row beyond 1024)."""
+    H, Hkv, d, B, S = 2, 1, 64, 64, 4
+    r, Nb = B // S, L // B
+    q, _, _ = gen.make_qkv(L, H, Hkv, d, gen.IID, 51)
+    kd = torch.zeros((L, Hkv, d), dtype=torch.bfloat16, device="cuda")
+    ws = rr.workspace(L, H, Hkv, d, B, S)
+    mass = torch.zeros((H, Nb, Nb), dtype=torch.float32, device="cuda")
+    count, idx = rr.search(to_dev(q), kd, B, S, tau, mass=mass, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+    count, idx, M = count.cpu().numpy(), idx.cpu().numpy(), mass.cpu().numpy()
+    check_mask_format(count, idx)
+    checked = 0
+    for h in range(H):
+        for I in range(Nb - 1):
+            assert np.all(M[h, I, :I] == M[h, I, 0]), (h, I)   # the ties are exact
+            # closed form: full block a = r * sum 1/(i+1), diagonal b = sum (i - I*r + 1)/(i+1)
+            i = np.arange(I * r, I * r + r, dtype=np.float64)
+            a, b = r * np.sum(1.0 / (i + 1)), np.sum((i - I * r + 1) / (i + 1))
+            total = I * a + b
+            k = next((k for k in range(1, I + 1) if k * a >= tau * total), None)
+            want = list(range(k)) if k is not None else list(range(I + 1))
+            share = (len(want) * a if k is not None else total) / total
+            if abs(share - tau) < 1e-6 or (k is not None and abs((k - 1) * a / total - tau) < 1e-6):
+                continue   # cut within rounding of tau: either side is right
+            assert count[h, I] == len(want), (h, I, count[h, I], len(want))
+            assert np.array_equal(idx[h, I, :count[h, I]], want), (h, I)
+            checked += 1
+    assert checked > 0.99 * H * (Nb - 1)
+
+
 def test_deterministic(rr):
     L, H, Hkv, d, B, S = 4096, 8, 2, 128, 128, 16
     q, k, v = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 5)
