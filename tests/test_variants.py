@@ -115,6 +115,49 @@ def test_flags_zero_is_rr_search(rr):
     assert torch.equal(torch.where(cols, i0, 0), torch.where(cols, i1, 0))
 
 
+def test_gqa_mask_long_rows_radix_path(rr):
+    """Rows longer than 1024 blocks (Nb = 2048) with one mask per GQA group: the
+    CTA-per-row Top-tau path writing each selection to both heads of a group.
+    Checked on sampled rows against the group mass the GPU selected on (the
+    heads' fp32 block masses summed in head order): every head of a group has
+    the same list, the list reaches tau of the row, dropping its lightest block
+    falls below tau, and no dropped block outweighs a kept one (equal masses
+    keep the lower J)."""
+    L, H, Hkv, d, B, S, tau = 131072, 4, 2, 64, 64, 16, 0.9
+    Nb = L // B
+    q, k, _ = gen.make_qkv(L, H, Hkv, d, gen.PLANTED_BAND, 61)
+    mass = torch.zeros((H, Nb, Nb), dtype=torch.float32, device="cuda")
+    ws = rr.workspace(L, H, Hkv, d, B, S, flags=GQA)
+    count, idx = rr.search_variant(to_dev(q), to_dev(k), B, S, tau, GQA, mass=mass, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+    count, idx = count.cpu().numpy(), idx.cpu().numpy()
+    check_mask_format(count, idx)
+    g = H // Hkv
+    rng = np.random.default_rng(62)
+    rows = sorted(set(rng.integers(1024, Nb - 1, 48).tolist()) | {1024, Nb - 2})
+    for kv in range(Hkv):
+        for I in rows:
+            per_head = mass[kv * g:(kv + 1) * g, I, :I + 1].cpu().numpy()
+            gm = per_head[0].copy()
+            for t in range(1, g):
+                gm = gm + per_head[t]                     # fp32, head order
+            c = count[kv * g, I]
+            kept = idx[kv * g, I, :c]
+            for t in range(1, g):
+                assert count[kv * g + t, I] == c and np.array_equal(idx[kv * g + t, I, :c], kept)
+            gm = gm.astype(np.float64)
+            total = gm.sum()
+            drop = np.setdiff1d(np.arange(I + 1), kept)
+            share = gm[kept].sum() / total
+            assert share >= tau - 1e-6, (kv, I, share)
+            assert share - gm[kept].min() / total < tau + 1e-6, (kv, I)
+            if drop.size:
+                assert gm[kept].min() >= gm[drop].max(), (kv, I)
+                tied = drop[gm[drop] == gm[kept].min()]
+                if tied.size:
+                    assert tied.min() > kept[gm[kept] == gm[kept].min()].max(), (kv, I)
+
+
 @pytest.mark.slow
 def test_sampled_keys_video64k_full_size(rr):
     """Sampled keys (and the GQA mask on top) on the full video workload
