@@ -4,8 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one pass of the whole hot path over one attention layer's synthetic
-inputs: key pooling, the round-robin sampled-score search, Top-tau selection and
-the block-sparse attention, through the C ABI.  Default workload: the 128K
+inputs: the round-robin sampled-score search, Top-tau selection and the
+block-sparse attention, through the C ABI.  Default workload: the 128K
 LLaMA-3.1-8B-shaped GQA layer (H=32, Hkv=8, d=128, L=131072, B=128, S=16,
 tau=0.95, planted sinks + local band).
 
@@ -297,10 +297,10 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     visited = int(count.sum().item())
     flops = block_flops(cfg, visited)
-    # pool, search, top-tau (one launch per row-length class: rows up to 256,
-    # 512 and 1024 blocks, and longer), attention
+    # search, top-tau (one launch per row-length class: rows up to 256, 512 and
+    # 1024 blocks, and longer), attention
     nb = cfg.L // cfg.B
-    gpu_launches = (3 + 1 + (nb > 256) + (nb > 512) + (nb > 1024)) * args.steps
+    gpu_launches = (2 + 1 + (nb > 256) + (nb > 512) + (nb > 1024)) * args.steps
 
     # dense baseline: the same attention kernel with every causal block on.  The
     # sparse and dense launches alternate, so that both see the same clocks (the
@@ -499,8 +499,9 @@ def run_sweep(args):
 
 
 def variant_name(flags: int) -> str:
-    """rr: the plain search; rot / sk / gqa: the sampling variants of rr_search_variant."""
-    parts = [n for bit, n in ((1, "rot"), (2, "sk"), (4, "gqa")) if flags & bit]
+    """rr: the plain search (sampled keys); rot / mk / gqa: the sampling variants of
+    rr_search_variant (rotation, stride-mean keys, one mask per GQA group)."""
+    parts = [n for bit, n in ((1, "rot"), (2, "mk"), (4, "gqa")) if flags & bit]
     return "+".join(parts) if parts else "rr"
 
 
@@ -522,7 +523,7 @@ def main():
                     help="per-config table instead of the contract line: every config and tau")
     ap.add_argument("--variants", default="0",
                     help="with --recall or --sweep: comma-separated sampling-variant flags (1 rotate, "
-                         "2 sampled keys, 4 GQA mask; 0 the plain search)")
+                         "2 stride-mean keys, 4 GQA mask; 0 the plain search)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("note: fewer than 3 warm-up steps requested", file=sys.stderr)

@@ -18,7 +18,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librr.so")
 
-RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT, RR_ESCRATCH = range(7)
+RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT, RR_ESCRATCH, RR_EMASK = range(8)
 
 # every symbol that include/rr.h declares
 EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status",
@@ -27,7 +27,7 @@ EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "
            "rr_workspace_size_host", "rr_attention_host")
 
 # sampling-variant flags of rr_search_variant (rr.h)
-VAR_ROTATE, VAR_SAMPLED_KEYS, VAR_GQA_MASK = 1, 2, 4
+VAR_ROTATE, VAR_MEAN_KEYS, VAR_GQA_MASK = 1, 2, 4
 
 
 class RRError(RuntimeError):
@@ -150,7 +150,7 @@ def search(q, k, B: int, S: int, tau: float, count=None, idx=None, mass=None, ws
 def search_variant(q, k, B: int, S: int, tau: float, flags: int, count=None, idx=None, mass=None, ws=None,
                    stream=None):
     """Pattern search with the sampling variants ``flags`` (VAR_ROTATE,
-    VAR_SAMPLED_KEYS, VAR_GQA_MASK, or-ed) -> (count, idx).  ``mass`` receives the
+    VAR_MEAN_KEYS, VAR_GQA_MASK, or-ed) -> (count, idx).  ``mass`` receives the
     per-head block masses."""
     L, H, Hkv, d = _shape(q, k)
     Nb = L // B

@@ -1,6 +1,7 @@
 // bsfa.cu — causal block-sparse FlashAttention forward over the selected
-// blocks (RRAttention abstract: "computing only half of the attention
-// blocks", "2.4x speedup at 128K"; Figure 2 stage 3; Figure 3a).
+// blocks (RRAttention page, Abstract: about half of the blocks computed and a
+// 2.4x speedup at 128K on the pages' workloads; Figure 2 caption: stage 3;
+// Figure 3 caption, panel a).
 //
 // One CTA per (head h, query block I), launched kv head by kv head, longest
 // rows first: a 128-row query tile (the B = 64 case
@@ -27,9 +28,10 @@
 // 3 MMA issuers (one thread each) for softmax groups 0 and 1, taking strict
 // turns by whole MMA brackets (warp 1 also owns the 512-column TMEM
 // allocation); warp 2 idle; warps 4-7 softmax group 0, warps 8-11 softmax
-// group 1.  The first warpgroup
-// gives registers back (setmaxnreg 48) so that the softmax groups can hold a
-// full 128-column score row (setmaxnreg 224): 128*48 + 256*224 <= 384*168.
+// group 1.  The first warpgroup gives registers back so that the softmax
+// groups can hold a full score row: setmaxnreg 56 / 224 at B = 128 and
+// 80 / 200 at B = 64, both within the launch's 384 * 168 registers
+// (128*56 + 256*224 = 64512, 128*80 + 256*200 = 61440).
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512);
 // P_x overwrites the last B/2 columns of S_x, so that the first half of the
 // scores is still there when a row's block has to be redone.
@@ -47,12 +49,6 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kStages = 4;
-
-// Every RR_EMU_EVERY-th exp2 pair of a non-diagonal block runs on the FMA pipe
-// (ex2_fma_x2) instead of MUFU; 0 keeps every exp2 on MUFU.
-#ifndef RR_EMU_EVERY
-#define RR_EMU_EVERY 0
-#endif
 
 template <int BN, int D>
 struct FaCfg {
@@ -84,9 +80,8 @@ struct FaCtrl {
 };
 
 // Exponentiate one row of scores into P = 2^(s*sl2 - m) (bf16, written to TMEM
-// at p_col) and return the row sum of P in fp32.  kEmu > 0 moves every kEmu-th
-// pair from MUFU to the FMA pipe (ex2_fma_x2).
-template <int BN, int kEmu>
+// at p_col) and return the row sum of P in fp32.
+template <int BN>
 __device__ __forceinline__ float exp_store(const float (&s)[BN], float sl2, float m_run, uint32_t p_col) {
   const uint64_t scale2 = f2pack(sl2, sl2);
   const uint64_t negm2 = f2pack(-m_run, -m_run);
@@ -100,14 +95,9 @@ __device__ __forceinline__ float exp_store(const float (&s)[BN], float sl2, floa
     for (int j = 0; j < 16; ++j) {
       const int jj = c * 16 + j;
       const uint64_t xp = fma2(f2pack(s[2 * jj], s[2 * jj + 1]), scale2, negm2);
-      uint64_t pp;
-      if (kEmu > 0 && (jj % (kEmu > 0 ? kEmu : 1)) == kEmu - 1) {
-        pp = ex2_fma_x2(xp);
-      } else {
-        float x0, x1;
-        f2unpack(xp, x0, x1);
-        pp = f2pack(ex2(x0), ex2(x1));
-      }
+      float x0, x1;
+      f2unpack(xp, x0, x1);
+      const uint64_t pp = f2pack(ex2(x0), ex2(x1));
       acc[j & 3] = add2(acc[j & 3], pp);
       float p0, p1;
       f2unpack(pp, p0, p1);
@@ -169,7 +159,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int h = kvh * g + r % g;
   const long long row_id = static_cast<long long>(h) * Nb + I;
   int cnt = count[row_id];
-  cnt = cnt < 0 ? 0 : (cnt > Nb ? Nb : cnt);
   const int32_t* list = idx + row_id * Nb;
 
   if (threadIdx.x == 0) {
@@ -195,13 +184,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(&ctl->tmem_base), 512);
     tmem_relinquish();
   }
+  // The row's block list, read coalesced into shared memory by every thread and
+  // checked against the mask format: count in [1, I+1], entries strictly
+  // ascending inside [0, I].  A list that breaks it (a key block above the
+  // diagonal would attend to future keys, one past Nb would read past the
+  // tensor) is not computed: the row's output is zero and the status word
+  // records the mask error with the row.
+  int bad = (cnt < 1 || cnt > I + 1) ? 1 : 0;
+  if (!bad) {
+    for (int t = threadIdx.x; t < cnt; t += kThreads) {
+      const int J = __ldg(list + t);
+      const int prev = t > 0 ? __ldg(list + t - 1) : -1;
+      if (J < 0 || J > I || J <= prev) bad = 1;
+      sList[t] = J;
+    }
+  }
   tc_fence_before();
-  __syncthreads();
+  bad = __syncthreads_or(bad);
   tc_fence_after();
+  if (bad) {
+    if (threadIdx.x == 0)
+      atomicCAS(status, 0u, kStatusMaskCode | (static_cast<unsigned>(row_id < (1 << 24) ? row_id : (1 << 24) - 1) << 8));
+    cnt = 0;
+  }
   const uint32_t tm = ctl->tmem_base;
   const Guard guard{&ctl->abort, status, limit_ns};
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 48;\n" ::: "memory");
+    if constexpr (BN == 128) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+    } else {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
+    }
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && cnt > 0) {
@@ -212,9 +225,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_expect_tx(qb, C::kQBytes);
       for (int a = 0; a < D / 64; ++a) tma_load_3d(smem_u32(sQ + a * 128 * 128), &mq, qb, a * 64, h, I * BN);
     }
-    // the block list, read coalesced into shared memory
-    for (int t = lane; t < cnt; t += 32) sList[t] = __ldg(list + t);
-    __syncwarp();
     if (lane == 0 && cnt > 0) {
       int k = 0;
       bool ok = true;
@@ -343,7 +353,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;\n" ::: "memory");
+    if constexpr (BN == 128) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 224;\n" ::: "memory");
+    } else {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
+    }
     // ------------------------------------------------------------ softmax groups
     const int x = (warp - 4) >> 2;              // group 0: warps 4-7, group 1: warps 8-11
     const int wq = warp & 3;                    // TMEM lane quarter
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_col = tm + lane_off + 256 + x * 128;
     const int n_a = (cnt + 1) >> 1, n_b = cnt >> 1;
     const int n_x = x == 0 ? n_a : n_b;
-    const bool diag_last = cnt > 0 && __ldg(list + cnt - 1) == I;
+    const bool diag_last = cnt > 0 && sList[cnt - 1] == I;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int u = 0; u < n_x; ++u) {
@@ -381,13 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // once, with no max pass: only when a row's block sum passes kSumLimit
       // (some score grew far above the running max) does that row take its
       // exact block max, rescale O and l, and redo the block.
-      auto expo = [&]() {
-        if constexpr (RR_EMU_EVERY == 0) {
-          return exp_store<BN, 0>(s, sl2, m_run, p_col);
-        } else {
-          return diag ? exp_store<BN, 0>(s, sl2, m_run, p_col) : exp_store<BN, RR_EMU_EVERY>(s, sl2, m_run, p_col);
-        }
-      };
+      auto expo = [&]() { return exp_store<BN>(s, sl2, m_run, p_col); };
       bool rescale = false;
       float alpha = 1.0f;
       if (u == 0) m_run = row_max<BN>(s) * sl2;
@@ -484,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 4; ++j) d4[j] = pk[j];
       }
     } else if (cnt == 0 && row < BN) {
-      // no block selected (not a mask rr_search produces): the row has no keys
+      // a row whose list broke the mask format: zero output (status recorded above)
       __nv_bfloat16* dst = o + ((static_cast<long long>(I) * BN + row) * H + h) * D;
       for (int c = x * (D / 2); c < (x + 1) * (D / 2); c += 8)
         *reinterpret_cast<uint4*>(dst + c) = make_uint4(0, 0, 0, 0);

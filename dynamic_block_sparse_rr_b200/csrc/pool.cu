@@ -1,5 +1,7 @@
-// pool.cu — stride-level key aggregation (RRAttention abstract: "stride-level
-// aggregation", O(L^2/S^2) search cost).  The S keys of stride j are averaged
+// pool.cu — stride-mean keys, the alternative reading of the search's key side
+// (RRAttention page, Abstract: scores gathered per stride at O(L^2/S^2) cost;
+// the pages do not say whether a stride's keys are sampled or averaged, and the
+// default search samples them).  The S keys of stride j are averaged
 // in fp32 (sequential order t = 0..S-1) and stored as a bf16 pair so that the
 // tensor-core search sees the mean to about 16 significant bits:
 //   hi = bf16_rn(mean), lo = bf16_rn(mean - hi).

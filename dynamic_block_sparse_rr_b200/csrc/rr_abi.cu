@@ -17,10 +17,11 @@ constexpr size_t kAlign = 256;
 
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-constexpr unsigned kVarAll = RR_VAR_ROTATE | RR_VAR_SAMPLED_KEYS | RR_VAR_GQA_MASK;
+constexpr unsigned kVarAll = RR_VAR_ROTATE | RR_VAR_MEAN_KEYS | RR_VAR_GQA_MASK;
 
-// Workspace regions (byte offsets).  With flags 0 only status, khi, klo and mass
-// are present, in that order (the rr_search layout).
+// Workspace regions (byte offsets).  With flags 0 only status and mass are
+// present (the rr_search layout); the pooled-key pair khi/klo only with
+// RR_VAR_MEAN_KEYS, the gathered rows only when rotating.
 struct Layout {
   size_t status, khi, klo, qs, ks, mass, gmass, total;
 };
@@ -28,7 +29,7 @@ struct Layout {
 Layout carve(int L, int H, int Hkv, int d, int B, int S, unsigned flags = 0) {
   Layout w;
   const size_t Ns = static_cast<size_t>(L / S), Nb = static_cast<size_t>(L / B);
-  const bool pooled = !(flags & RR_VAR_SAMPLED_KEYS);
+  const bool pooled = (flags & RR_VAR_MEAN_KEYS) != 0;
   const bool rotate = (flags & RR_VAR_ROTATE) != 0;
   const size_t kbar = pooled ? round_up(Ns * Hkv * d * 2) : 0;
   const size_t gathered = round_up(Ns * H * d * 2);
@@ -65,7 +66,7 @@ rr_status enqueue_search(const void* q, const void* k, int L, int H, int Hkv, in
                          unsigned flags, int head0, int32_t* count, int32_t* idx, float* mass, uint8_t* ws,
                          const Layout& w, const rr::DeviceGuardArgs& g, cudaStream_t s) {
   float* m = mass ? mass : reinterpret_cast<float*>(ws + w.mass);
-  const bool rotate = (flags & RR_VAR_ROTATE) != 0, sampled = (flags & RR_VAR_SAMPLED_KEYS) != 0;
+  const bool rotate = (flags & RR_VAR_ROTATE) != 0, sampled = (flags & RR_VAR_MEAN_KEYS) == 0;
   const int g_heads = H / Hkv;
   rr::SearchSources src{q, ws + w.khi, ws + w.klo, 0, 0, head0};
   if (rotate) {
@@ -338,6 +339,7 @@ rr_status rr_check_status(void* workspace, void* stream) {
   if (cudaMemcpyAsync(&host, workspace, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return RR_ECUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return RR_ECUDA;
   if ((host & 0xFFu) == rr::kStatusTimeoutCode) return RR_ETIMEOUT;
+  if ((host & 0xFFu) == rr::kStatusMaskCode) return RR_EMASK;
   return host == 0 ? RR_OK : RR_ECUDA;
 }
 
@@ -356,6 +358,7 @@ const char* rr_status_string(rr_status s) {
     case RR_ECUDA: return "CUDA error";
     case RR_ETIMEOUT: return "device-side wait timed out";
     case RR_ESCRATCH: return "shape needs more scratch than rr_search_static's 32 MiB array";
+    case RR_EMASK: return "block list outside the mask format (row not computed)";
   }
   return "unknown status";
 }

@@ -82,6 +82,9 @@ cudaError_t set_smem_limit_once(Kernel kernel, int bytes, std::atomic<uint64_t>&
 
 // Low byte of the workspace status word when a device-side wait ran out.
 constexpr unsigned kStatusTimeoutCode = 5u;
+// Low byte of the workspace status word when the attention kernel met a block
+// list outside the mask format (bits 8..31: the row h*Nb + I, saturated).
+constexpr unsigned kStatusMaskCode = 7u;
 
 // Largest Nb = L/B the kernels accept (bounded by the on-chip list / sort buffers).
 constexpr int kMaxBlocks = 4096;

@@ -1,17 +1,18 @@
 // search.cu — the round-robin sampled-score pass and block-mass aggregation
-// (RRAttention abstract: "head round-robin (RR) sampling", "stride-level
-// aggregation", "O(L^2/S^2)"; Figure 2 stages 1 and 2).
+// (RRAttention page, Abstract: per-head round-robin sampling, scores gathered
+// per stride, a search cost of O(L^2/S^2); Figure 2 caption: stages 1 and 2).
 //
-// Head h samples, in stride i, the query at position i*S + (h mod S).  These
-// Ns = L/S real queries are scored against the Ns stride-pooled keys of the
-// head's kv group: s[i, j] = q_i . kbar_j / sqrt(d) for j <= i.  That is a
-// causal "mini attention" of length Ns, computed in 128 x 128 tiles:
+// Head h samples, in stride i, position p(h, i) = i*S + (h mod S).  Its Ns = L/S
+// sampled queries are scored against the Ns keys at the same positions of its
+// kv head: s[i, j] = q_p(h,i) . k_p(h,j) / sqrt(d) for j <= i.  That is a causal
+// attention over the head's strided subsequence, computed in 128 x 128 tiles:
 //
 //   * one CTA per (head, tile of 128 sampled rows); heavier tiles launch first;
-//   * the sampled rows are read zero-copy through a 4D TMA view of q
-//     (d, H, S, Ns), so no sampled copy is ever materialised;
-//   * S = Qs Kbar^T runs on tcgen05 (bf16 in, fp32 accumulate in TMEM) as two
-//     MMA chains, Qs*Khi^T + Qs*Klo^T, so the pooled keys enter at ~16 bits;
+//   * the sampled rows and keys are read zero-copy through 4D TMA views
+//     (d, heads, S, Ns), so no sampled copy is ever materialised;
+//   * S = Qs Ks^T runs on tcgen05 (bf16 in, fp32 accumulate in TMEM); with the
+//     stride-mean keys of the alternative reading it is two MMA chains,
+//     Qs*Khi^T + Qs*Klo^T, so the pooled keys enter at ~16 bits;
 //   * pass 1 walks the row's key tiles for the row log-sum-exp (online), pass 2
 //     recomputes the identical scores, forms P = exp(s - lse) and sums P over
 //     the r x r (sampled row, stride) pairs of each B x B block with warp

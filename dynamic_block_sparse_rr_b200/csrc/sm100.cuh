@@ -367,38 +367,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
-// 2^x on the FMA pipe, for x >= -125 (smaller x is clamped): x = j + f with
-// j = round(x) (1.5 * 2^23 rounding trick), f in [-1/2, 1/2]; 2^f from a
-// degree-3 polynomial fitted by Remez exchange for minimum relative error on
-// [-1/2, 1/2] (fit_exp2.py: max relative error 7.5e-5, far below the bf16
-// rounding of P); 2^j is added to the exponent field.
-__device__ __forceinline__ float ex2_fma(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
-  p = fmaf(p, f, 6.932609677e-01f);
-  p = fmaf(p, f, 9.999280572e-01f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// ex2_fma on a packed pair (same arithmetic, f32x2 instructions).
-__device__ __forceinline__ uint64_t ex2_fma_x2(uint64_t xp) {
-  float x0, x1;
-  f2unpack(xp, x0, x1);
-  const uint64_t xc = f2pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t t = add2(xc, f2pack(12582912.0f, 12582912.0f));
-  const uint64_t f = fma2(add2(t, f2pack(-12582912.0f, -12582912.0f)), f2pack(-1.0f, -1.0f), xc);
-  uint64_t p = fma2(f2pack(5.517166853e-02f, 5.517166853e-02f), f, f2pack(2.426111251e-01f, 2.426111251e-01f));
-  p = fma2(p, f, f2pack(6.932609677e-01f, 6.932609677e-01f));
-  p = fma2(p, f, f2pack(9.999280572e-01f, 9.999280572e-01f));
-  float p0, p1, t0, t1;
-  f2unpack(p, p0, p1);
-  f2unpack(t, t0, t1);
-  return f2pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
-                __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
-}
-
 // Two fp32 -> packed bf16x2 (lo in bits 0-15), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -1,6 +1,6 @@
-// topk.cu — adaptive Top-tau block selection with static protection of the
-// last query block (RRAttention abstract: "adaptive Top-tau selection"; TL;DR:
-// "Top-tau block selection and a static protection of the last query block").
+// topk.cu — adaptive Top-tau block selection with the last query block always
+// kept (RRAttention page, Abstract: the adaptive Top-tau cut; TL;DR: Top-tau
+// selection plus a fixed protection of the final query block).
 //
 // The kept set of row (h, I) is the shortest prefix, in (mass descending, J
 // ascending) order, of its I+1 block masses whose sum reaches tau * (row

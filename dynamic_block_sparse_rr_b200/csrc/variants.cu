@@ -3,7 +3,8 @@
 // stands for the keys of a stride, and whether GQA heads share one mask):
 //
 //   gather_rotated: the rows at the rotating offsets p(h, i) = i*S + (h + i) mod S,
-//     gathered into a dense [Ns, H, d] array the search reads with plain 3D tiles.
+//     gathered into a dense [Ns, H, d] array the search reads with plain 3D tiles
+//     (queries, and keys unless the stride-mean keys are asked for).
 //     HBM-bound: reads and writes Ns*H*d*2 bytes; one thread per 16 bytes,
 //     consecutive threads on consecutive addresses of one row.
 //   group_mass: the block masses of the g query heads of a kv head summed, in

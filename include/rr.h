@@ -1,12 +1,13 @@
 /*
  * rr.h — C ABI of the B200 (sm_100a) RRAttention prefill operator.
  *
- * The operator is the one described in "RRAttention: Dynamic Block Sparse
- * Attention via Per-Head Round-Robin Shifts for Long-Context Inference"
- * (Abstract and TL;DR; Figure 2 caption for the three stages): a head
- * round-robin strided pattern search that selects, per query block, an
- * adaptive Top-tau set of key blocks (the last query block kept dense),
- * followed by causal block-sparse attention over the selected blocks.
+ * The operator is the one described on the pages of "RRAttention: Dynamic
+ * Block Sparse Attention via Per-Head Round-Robin Shifts for Long-Context
+ * Inference" (sciencestack page: Abstract, TL;DR, Figure 2 caption for the
+ * three stages): a strided pattern search in which each head samples one
+ * position per stride, the position shifting from head to head, that picks per
+ * query block an adaptive Top-tau set of key blocks (the last query block kept
+ * dense), followed by causal block-sparse attention over the selected blocks.
  *
  * Notation: H query heads, Hkv kv heads (H % Hkv == 0, g = H/Hkv), head dim d,
  * sequence length L, block size B, stride S; Ns = L/S, Nb = L/B, r = B/S.
@@ -47,20 +48,23 @@ typedef enum {
   RR_EALIGN = 3,
   RR_ECUDA = 4,
   RR_ETIMEOUT = 5,
-  RR_ESCRATCH = 6   /* rr_search_static only: the shape needs more than its static scratch */
+  RR_ESCRATCH = 6,  /* rr_search_static only: the shape needs more than its static scratch */
+  RR_EMASK = 7      /* rr_sparse_attn: a block list outside the mask format (row not computed) */
 } rr_status;
 
 /* Bytes of device workspace that rr_search / rr_sparse_attn / rr_attention
- * need for this shape (pooled keys, block masses, status word).  The same
+ * need for this shape (status word and block masses [H, Nb, Nb] fp32).  The same
  * workspace may be reused by consecutive calls on one stream. */
 rr_status rr_workspace_size(int L, int H, int Hkv, int d, int B, int S, size_t* bytes);
 
-/* Pattern search (Abstract: head round-robin sampling, stride-level
- * aggregation, adaptive Top-tau; TL;DR: static protection of the last query
- * block; Figure 2 stages 1 and 2).
- *   Sampling: head h samples, in stride i, the query at i*S + (h mod S).
- *   Keys:     the S keys of stride j are averaged (fp32, kept as a bf16 pair).
- *   Scores:   s[h,i,j] = q . kbar[j] / sqrt(d) for j <= i, softmax per row.
+/* Pattern search (RRAttention page, Abstract: head round-robin sampling with
+ * scores aggregated per stride and an adaptive Top-tau cut; TL;DR: the last
+ * query block is always kept; Figure 2 caption: stages 1 and 2).
+ *   Sampling: head h samples, in stride i, position p(h,i) = i*S + (h mod S),
+ *             on both sides: its query rows and, on its kv head, its keys.
+ *   Scores:   s[h,i,j] = q[p(h,i),h] . k[p(h,j),h/g] / sqrt(d) for j <= i,
+ *             softmax per sampled row (a causal attention over the head's
+ *             strided subsequence, L/S long).
  *   Mass:     summed over the r x r (row, stride) pairs of block (I, J).
  *   Top-tau:  per row I < Nb-1, blocks in (mass desc, J asc) order, shortest
  *             prefix whose share of the row's mass is >= tau (tau >= 1: all).
@@ -79,15 +83,15 @@ rr_status rr_search(const void* q, const void* k, int L, int H, int Hkv, int d, 
                     size_t workspace_bytes, void* stream);
 
 /* Sampling variants of the pattern search.  The pages fix the head rotation of
- * the sampled offset and the stride-level aggregation of keys, but leave open
- * three choices, each selectable here (flags may be combined; 0 = rr_search):
+ * the sampled offset and the stride-level scoring, but leave open three
+ * choices, each selectable here (flags may be combined; 0 = rr_search):
  *   RR_VAR_ROTATE        the offset rotates across strides as well as heads:
- *                        head h samples, in stride i, the query at
- *                        i*S + ((h + i) mod S).
- *   RR_VAR_SAMPLED_KEYS  the key side of stride j is the single key at the
- *                        head's own sampled position of that stride (the same
- *                        rule as its queries) instead of the mean of the S
- *                        keys: same O(L^2/S^2) cost, no averaging.
+ *                        head h samples, in stride i, position
+ *                        i*S + ((h + i) mod S), on both sides.
+ *   RR_VAR_MEAN_KEYS     the key side of stride j is the mean of the stride's S
+ *                        keys (fp32, kept as a bf16 hi/lo pair) instead of the
+ *                        key at the head's own sampled position: same
+ *                        O(L^2/S^2) cost, per-token structure averaged away.
  *   RR_VAR_GQA_MASK      one mask per GQA group: the Top-tau selection runs
  *                        on the sum of the block masses of the H/Hkv query
  *                        heads of a kv head, and every head of the group
@@ -95,11 +99,12 @@ rr_status rr_search(const void* q, const void* k, int L, int H, int Hkv, int d, 
  * Scores, block mass, Top-tau and the last-row protection are those of
  * rr_search.  Out: count [H,Nb], idx [H,Nb,Nb]; mass (optional) receives the
  * per-head block mass [H,Nb,Nb] before any group sum.  The workspace is sized
- * by rr_workspace_size_variant with the same flags (it holds the gathered
- * rows [L/S, H, d] bf16 when rotating, the group masses [Hkv, Nb, Nb] fp32
- * with RR_VAR_GQA_MASK).  Unknown flag bits: RR_EINVAL. */
+ * by rr_workspace_size_variant with the same flags (it holds the pooled keys
+ * [L/S, Hkv, d] x 2 bf16 with RR_VAR_MEAN_KEYS, the gathered rows
+ * [L/S, H, d] bf16 when rotating, the group masses [Hkv, Nb, Nb] fp32 with
+ * RR_VAR_GQA_MASK).  Unknown flag bits: RR_EINVAL. */
 #define RR_VAR_ROTATE 1u
-#define RR_VAR_SAMPLED_KEYS 2u
+#define RR_VAR_MEAN_KEYS 2u
 #define RR_VAR_GQA_MASK 4u
 rr_status rr_workspace_size_variant(int L, int H, int Hkv, int d, int B, int S, unsigned flags,
                                     size_t* bytes);
@@ -107,14 +112,20 @@ rr_status rr_search_variant(const void* q, const void* k, int L, int H, int Hkv,
                             float tau, unsigned flags, int32_t* count, int32_t* idx, float* mass,
                             void* workspace, size_t workspace_bytes, void* stream);
 
-/* Causal block-sparse attention over a block mask (Abstract: "computing only
- * half of the attention blocks"; Figure 2 stage 3).  Query q of block I, head
+/* Causal block-sparse attention over a block mask (RRAttention page, Abstract:
+ * only the selected blocks are computed; Figure 2 caption: stage 3).  Query q of block I, head
  * h, attends with scale 1/sqrt(d) to every key k <= q of the blocks listed for
  * (h, I); kv head = h / (H/Hkv).  fp32 softmax and accumulation, bf16 output.
- * In:  q, k, v bf16 (device), count/idx as produced by rr_search (any valid
- *      mask in the format above is accepted; entries are not range-checked on
- *      the device beyond the debug checks of the kernel).
- * Out: o [L,H,d] bf16 (device, caller-owned). */
+ * In:  q, k, v bf16 (device), count/idx as produced by rr_search (any mask in
+ *      the format above is accepted).
+ * Out: o [L,H,d] bf16 (device, caller-owned).
+ * Mask check: the kernel checks every row it reads against the format (count
+ * in [1, I+1], entries strictly ascending inside [0, I]).  A row that breaks it
+ * is not computed (its B output rows of head h are written as zeros) and the
+ * workspace status word records RR_EMASK with the first such row seen;
+ * rr_check_status returns RR_EMASK.  Other rows are unaffected.  The check
+ * reads only the count entry and the first count entries of the row's list,
+ * so a count outside [1, I+1] is rejected without reading the list. */
 rr_status rr_sparse_attn(const void* q, const void* k, const void* v, int L, int H, int Hkv, int d,
                          int B, const int32_t* count, const int32_t* idx, void* o, void* workspace,
                          size_t workspace_bytes, void* stream);
@@ -172,8 +183,8 @@ rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int 
                            void* stream);
 
 /* Synchronises `stream`, returns the device-side status recorded since the
- * last rr_* call that started on this workspace (RR_OK or RR_ETIMEOUT), and
- * RR_ECUDA if the stream reports an error. */
+ * last rr_* call that started on this workspace (RR_OK, RR_ETIMEOUT or
+ * RR_EMASK), and RR_ECUDA if the stream reports an error. */
 rr_status rr_check_status(void* workspace, void* stream);
 
 /* Sets the bound, in nanoseconds, of every device-side wait of later launches

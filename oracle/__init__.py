@@ -5,45 +5,50 @@ CPU-baseline leg of ``bench.py`` may import this module.  It shares no code with
 the CUDA path (``dynamic_block_sparse_rr_b200``) and the CUDA path never calls it.
 
 It restates, plainly and slowly, what the method computes.  The source is the
-RRAttention abstract and TL;DR ("RRAttention: Dynamic Block Sparse Attention via
-Per-Head Round-Robin Shifts for Long-Context Inference", sciencestack.ai page:
-Abstract, TL;DR, Figure 2 and Figure 3 captions; the same abstract on the
-taxoreview, paperdot and fugumt pages).  The pages carry no equations and no
-algorithm box, so every definition below is the plainest reading of that text.
-The readings:
+RRAttention pages (sciencestack.ai page of "RRAttention: Dynamic Block Sparse
+Attention via Per-Head Round-Robin Shifts for Long-Context Inference": Abstract,
+TL;DR, Figure 2 and Figure 3 captions; the taxoreview, paperdot and fugumt pages
+repeat the same abstract).  The pages carry no equations and no algorithm box,
+so every definition below is the plainest reading of that text, stated in our
+own words.  The readings:
 
-R1  Sampling ("rotating query sampling positions across attention heads within
-    each stride"; title: "Per-Head Round-Robin Shifts").  Head h samples, in
-    stride i, the query at position p(h, i) = i*S + (h mod S).  The shift is
-    fixed per head; it does not rotate across strides.
-R2  Stride-level keys ("stride-level aggregation", cost O(L^2/S^2)).  The keys
-    of stride j are reduced to their mean, Kbar[j] = (1/S) sum_{t<S} K[j*S+t].
-    The O(L^2/S^2) cost needs the key side reduced by S as well; the mean keeps
-    every key's contribution while the queries stay real, unpooled rows
-    ("query independence").                                   [parity unpinned]
-R3  Scores.  s[h,i,j] = Qs[h,i] . Kbar[j, h/g] / sqrt(d) for stride-causal j <= i
-    (the diagonal stride is included, so a row is never empty).
-                                                              [parity unpinned]
+R1  Sampling (Abstract: the sampled query position rotates from head to head
+    inside every stride; title: per-head round-robin shifts).  Head h samples,
+    in stride i, the position p(h, i) = i*S + (h mod S).  The shift is fixed per
+    head; it does not rotate across strides.
+R2  Stride-level keys (Abstract: the method is a sampling strategy, and that
+    sampling is what lowers the search cost to O(L^2/S^2)).  Head h reads the
+    key side of stride j at its own sampled position too: the key at
+    p(h, j) = j*S + (h mod S) of its kv head.  Every score is then the logit of a
+    real (query, key) token pair, and each head's search is causal attention
+    over its own strided subsequence.  Across S heads every offset of every
+    stride is seen.                                           [parity unpinned
+    for S > 1 beyond the pins listed below]
+R3  Scores.  s[h,i,j] = Q[p(h,i), h] . K[p(h,j), h/g] / sqrt(d) for stride-causal
+    j <= i (the diagonal stride is included, so a row is never empty).
 R4  Each sampled row is a softmax over its j <= i.
-R5  Block mass ("aggregates the scores to BxB blocks").  A query block I holds
-    the r = B/S sampled rows i with i*S in I, a key block J the r strides j
-    with j*S in J.  M[h,I,J] = sum_{i in I} sum_{j in J} P[h,i,j], normalised
-    per row: m[h,I,J] = M[h,I,J] / sum_{J' <= I} M[h,I,J'].
-R6  Adaptive Top-tau ("smallest set of key blocks whose normalised mass reaches
-    tau").  For each row I < Nb-1: order J in [0, I] by (m descending, J
-    ascending), keep the shortest prefix whose running sum is >= tau.  tau >= 1
-    keeps every J <= I.
-R7  Static protection of the last query block (TL;DR): the last row I = Nb-1
-    keeps every J <= Nb-1, for every tau.  No other block is forced.
-R8  Block-sparse causal attention ("computing only half of the attention
-    blocks").  Query q in block I attends, with softmax scale 1/sqrt(d), to
-    every key k <= q that lies in a selected block of row I.
-V1-V3 Variants the pages leave open (off by default): V1 rotates the sampled
-    offset across strides too, p(h, i) = i*S + ((h + i) mod S); V2 takes the key
-    side of stride j as the single key at the head's offset instead of the
-    stride mean (same O(L^2/S^2) cost, no blurring of per-token structure); V3
-    keeps one mask per GQA group, selecting on the summed block mass of the
-    group's heads.                                            [parity unpinned
+R5  Block mass (Abstract: stride-level scores aggregated to B x B blocks;
+    Figure 2, stages 1-2).  A query block I holds the r = B/S sampled rows i
+    with i*S in I, a key block J the r strides j with j*S in J.
+    M[h,I,J] = sum_{i in I} sum_{j in J} P[h,i,j], normalised per row:
+    m[h,I,J] = M[h,I,J] / sum_{J' <= I} M[h,I,J'].
+R6  Adaptive Top-tau (Abstract; TL;DR).  For each row I < Nb-1: order J in
+    [0, I] by (m descending, J ascending), keep the shortest prefix whose
+    running sum is >= tau (the selected share reaches tau).  tau >= 1 keeps
+    every J <= I.
+R7  The last query block is protected (TL;DR): row I = Nb-1 keeps every
+    J <= Nb-1, for every tau.  No other block is forced.
+R8  Block-sparse causal attention (Abstract: only the selected blocks, about
+    half of them on the pages' workloads, are computed).  Query q in block I
+    attends, with softmax scale 1/sqrt(d), to every key k <= q that lies in a
+    selected block of row I.
+V1-V3 Alternatives the pages leave open (off by default): V1 rotates the
+    sampled offset across strides too, p(h, i) = i*S + ((h + i) mod S), on both
+    sides; V2 (mean_keys) replaces the sampled key of stride j by the mean of
+    the stride's S keys, Kbar[j] = (1/S) sum_{t<S} K[j*S+t], which costs the
+    same O(L^2/S^2) but blurs per-token structure; V3 keeps one mask per GQA
+    group, selecting on the summed block mass of the group's heads.
+                                                              [parity unpinned
     beyond the invariants in tests/test_oracle.py]
 R9  Mask comparison band (tolerance of the operator's specification): a block
     is near-threshold when the running sum just before or just after it, in
@@ -55,8 +60,10 @@ fp64 (tau = 1 and arbitrary block masks); R1-R5 at S = 1 against the exact
 full-attention block mass from the attention matrix that scaled_dot_product_
 attention returns; R3-R5 with all-zero keys against the closed form
 P[i,j] = 1/(i+1) (a hand-derived fixture in the Figure 2 configuration S=4,
-B=8); R6 against brute-force subset enumeration; R7 by inspection of every row.
-R2 and R3 for S > 1 have no pin beyond those reductions: "parity unpinned".
+B=8); R2 by planted keys that only the head's own offset on its own kv head
+sees; R6 against brute-force subset enumeration; R7 by inspection of every row.
+That the paper samples the key side this way, rather than pooling it, is a
+reading: "parity unpinned" for S > 1 against the paper itself.
 
 All arithmetic is float64.  Inputs are the bf16 values both paths receive,
 widened exactly (callers may pass them as float32 or float64 arrays; every
@@ -85,38 +92,39 @@ def rotated_positions(L: int, H: int, S: int) -> np.ndarray:
     return np.stack([i * S + (h + i) % S for h in range(H)])
 
 
-# ------------------------------------------------------------ R2 stride keys
+# ------------------------------------------------------- V2 stride-mean keys
 def pool_keys(K: np.ndarray, S: int) -> np.ndarray:
-    """Kbar[j, kv, :] = mean over the S keys of stride j (R2).  K: [L, Hkv, d]."""
+    """Kbar[j, kv, :] = mean over the S keys of stride j (V2).  K: [L, Hkv, d]."""
     L, Hkv, d = K.shape
     return K.astype(np.float64).reshape(L // S, S, Hkv, d).mean(axis=1)
 
 
 # ------------------------------------------------------- R3-R5 block masses
 def block_mass(Q: np.ndarray, K: np.ndarray, B: int, S: int, row_chunk: int = 2048,
-               rotate: bool = False, sampled_keys: bool = False) -> np.ndarray:
-    """Unnormalised block mass M[h, I, J] (R3-R5), zero above the diagonal.
+               rotate: bool = False, mean_keys: bool = False) -> np.ndarray:
+    """Unnormalised block mass M[h, I, J] (R2-R5), zero above the diagonal.
 
     Q: [L, H, d], K: [L, Hkv, d].  Returns [H, Nb, Nb] float64.
-    Variants (off by default): rotate -> V1 query positions; sampled_keys -> V2,
-    the key side of stride j is the single key at the head's own offset in that
-    stride (the same rule as its queries) instead of the stride mean.
+    Head h scores its sampled queries against the key at its own sampled
+    position of every stride (R2).  Alternatives (off by default): rotate -> V1
+    positions on both sides; mean_keys -> V2, the key side of stride j is the
+    mean of the stride's S keys.
     """
     L, H, d = Q.shape
     Hkv = K.shape[1]
     g = H // Hkv
     Ns, Nb, r = L // S, L // B, B // S
-    Kbar = None if sampled_keys else pool_keys(K, S)
+    Kbar = pool_keys(K, S) if mean_keys else None
     pos = rotated_positions(L, H, S) if rotate else sampled_positions(L, H, S)
     scale = 1.0 / math.sqrt(d)
     M = np.zeros((H, Nb, Nb), dtype=np.float64)
     step = max(r, (row_chunk // r) * r)
     for h in range(H):
         Qs = Q[pos[h], h, :].astype(np.float64)  # [Ns, d] real sampled queries
-        if sampled_keys:
-            Kb = K[pos[h], h // g, :].astype(np.float64)   # [Ns, d] one real key per stride
+        if mean_keys:
+            Kb = Kbar[:, h // g, :]                  # [Ns, d] stride means (V2)
         else:
-            Kb = Kbar[:, h // g, :]                  # [Ns, d]
+            Kb = K[pos[h], h // g, :].astype(np.float64)   # [Ns, d] one real key per stride (R2)
         for a in range(0, Ns, step):
             b = min(Ns, a + step)
             s = (Qs[a:b] @ Kb[:b].T) * scale     # rows i in [a,b), strides j < b
@@ -181,10 +189,10 @@ def select(m: np.ndarray, tau: float):
 
 
 def rr_search(Q: np.ndarray, K: np.ndarray, B: int, S: int, tau: float, rotate: bool = False,
-              sampled_keys: bool = False, gqa_mask: bool = False):
+              mean_keys: bool = False, gqa_mask: bool = False):
     """The pattern search: returns (count, idx, m) with m the normalised block mass
     (of the GQA group when gqa_mask)."""
-    M = block_mass(Q, K, B, S, rotate=rotate, sampled_keys=sampled_keys)
+    M = block_mass(Q, K, B, S, rotate=rotate, mean_keys=mean_keys)
     if gqa_mask:
         M = group_mass(M, K.shape[1])
     m = normalise_mass(M)
@@ -239,9 +247,9 @@ def sparse_attention(Q, K, V, count, idx, B: int, rows=None) -> np.ndarray:
 
 # ------------------------------------------------ mask diagnostics (recall)
 def exact_block_mass(Q, K, B: int) -> np.ndarray:
-    """Exact full-attention block mass: the R3-R5 definitions at S = 1, where every
-    query is sampled and every key is its own stride (pinned against the attention
-    matrix of torch's scaled_dot_product_attention)."""
+    """Exact full-attention block mass: the R2-R5 definitions at S = 1, where every
+    query and every key is sampled (pinned against the attention matrix of
+    torch's scaled_dot_product_attention)."""
     return block_mass(Q, K, B, 1)
 
 

@@ -33,7 +33,7 @@ def test_exports_every_declared_symbol(rr):
 
 
 def test_status_strings(rr):
-    for code in range(6):
+    for code in range(8):
         s = rr.status_string(code)
         assert isinstance(s, str) and s
     assert rr.status_string(0) == "ok"
@@ -72,7 +72,7 @@ def test_workspace_size_validation(rr, args, code):
     assert c == code
     if code == 0:
         L, H, Hkv, d, B, S = args
-        assert n >= H * (L // B) ** 2 * 4 + 2 * (L // S) * Hkv * d * 2
+        assert n >= H * (L // B) ** 2 * 4
 
 
 def test_search_rejects_before_any_launch(rr):
@@ -132,12 +132,12 @@ def test_variant_workspace_sizes(rr):
     Ns, Nb = L // S, L // B
     assert _ws_var(L, H, Hkv, d, B, S, 0) == _ws(L, H, Hkv, d, B, S)
     base = _ws_var(L, H, Hkv, d, B, S, 0)[1]
-    # sampled keys drop the pooled (hi, lo) pair
-    assert _ws_var(L, H, Hkv, d, B, S, rr.VAR_SAMPLED_KEYS)[1] == base - 2 * Ns * Hkv * d * 2
-    # rotation adds the gathered queries, and the gathered keys with sampled keys
-    assert _ws_var(L, H, Hkv, d, B, S, rr.VAR_ROTATE)[1] == base + Ns * H * d * 2
-    assert (_ws_var(L, H, Hkv, d, B, S, rr.VAR_ROTATE | rr.VAR_SAMPLED_KEYS)[1]
-            == base - 2 * Ns * Hkv * d * 2 + 2 * Ns * H * d * 2)
+    # stride-mean keys add the pooled (hi, lo) pair
+    assert _ws_var(L, H, Hkv, d, B, S, rr.VAR_MEAN_KEYS)[1] == base + 2 * Ns * Hkv * d * 2
+    # rotation adds the gathered queries and the gathered keys (sampled keys)
+    assert _ws_var(L, H, Hkv, d, B, S, rr.VAR_ROTATE)[1] == base + 2 * Ns * H * d * 2
+    assert (_ws_var(L, H, Hkv, d, B, S, rr.VAR_ROTATE | rr.VAR_MEAN_KEYS)[1]
+            == base + 2 * Ns * Hkv * d * 2 + Ns * H * d * 2)
     # the GQA mask adds the group masses
     assert _ws_var(L, H, Hkv, d, B, S, rr.VAR_GQA_MASK)[1] == base + Hkv * Nb * Nb * 4
     assert _ws_var(L, H, Hkv, d, B, S, 8)[0] == rr.RR_EINVAL
@@ -148,7 +148,7 @@ def test_search_variant_rejects_before_any_launch(rr):
     lib = rr.lib()
     g = 1 << 20
     L, H, Hkv, d, B, S = 1024, 4, 2, 64, 64, 4
-    flags = rr.VAR_ROTATE | rr.VAR_SAMPLED_KEYS | rr.VAR_GQA_MASK
+    flags = rr.VAR_ROTATE | rr.VAR_MEAN_KEYS | rr.VAR_GQA_MASK
     _, n = _ws_var(L, H, Hkv, d, B, S, flags)
 
     def call(flags=flags, q=g, nws=n, tau=0.9):

@@ -343,8 +343,49 @@ def test_sampled_keys_equal_mean_keys_when_strides_are_constant():
     K = np.repeat(_rand((L // S, Hkv, d), 61), S, axis=0)       # keys constant inside each stride
     for rotate in (False, True):
         a = oracle.block_mass(Q, K, B, S, rotate=rotate)
-        b = oracle.block_mass(Q, K, B, S, rotate=rotate, sampled_keys=True)
+        b = oracle.block_mass(Q, K, B, S, rotate=rotate, mean_keys=True)
         assert np.max(np.abs(a - b)) < 1e-12
+
+
+@pytest.mark.parametrize("rotate", [False, True])
+def test_sampled_keys_take_the_heads_own_offset(rotate):
+    """Sampled keys (R2): head h scores its sampled queries against the single key
+    at its own sampled position of every stride, on its own kv head h // g.
+
+    Every key is zero except one per query head: head h's key at its own offset
+    in stride j_h (a distinct stride per head) on kv head h // g, of size
+    30*sqrt(d) along e_0, and every query is e_0.  Head h then sees one logit of
+    30 (at stride j_h) and zeros elsewhere, so each of its sampled rows i >= j_h
+    puts all but i*e^-30 of its probability on stride j_h: the normalised mass of
+    key block j_h // r is 1 to within 1e-9 in every row whose first sampled row
+    is at or past j_h.  A key read at another offset (the next head's), from
+    another kv head, or averaged over the stride spreads that mass."""
+    L, H, Hkv, d, B, S = 512, 4, 2, 16, 32, 8
+    r, Nb, Ns = B // S, L // B, L // S
+    g = H // Hkv
+    Q = np.zeros((L, H, d))
+    Q[:, :, 0] = 1.0
+    K = np.zeros((L, Hkv, d))
+    j_of = {h: 9 + 11 * h for h in range(H)}                 # 9, 20, 31, 42: distinct blocks 2, 5, 7, 10
+    for h in range(H):
+        j = j_of[h]
+        off = (h + j) % S if rotate else h % S
+        K[j * S + off, h // g, 0] = 30.0 * math.sqrt(d)
+    m = oracle.normalise_mass(oracle.block_mass(Q, K, B, S, rotate=rotate))
+    for h in range(H):
+        Jh = j_of[h] // r
+        rows = [I for I in range(Nb) if I * r >= j_of[h]]
+        assert rows and len(rows) >= 4
+        for I in rows:
+            assert m[h, I, Jh] > 1.0 - 1e-9, (h, I, m[h, I, Jh])
+        # rows wholly before the planted stride see only zero keys: uniform 1/(i+1)
+        for I in range(Nb):
+            if (I + 1) * r - 1 < j_of[h]:
+                want = np.zeros(Nb)
+                for i in range(I * r, (I + 1) * r):
+                    for j in range(i + 1):
+                        want[j // r] += 1.0 / (i + 1)
+                assert np.allclose(m[h, I], want / r, atol=1e-12)
 
 
 def test_variants_at_stride_one_are_exact():
@@ -352,8 +393,8 @@ def test_variants_at_stride_one_are_exact():
     Q, K = _rand((L, H, d), 62), _rand((L, Hkv, d), 63)
     ref = oracle.block_mass(Q, K, B, 1)
     for rotate in (False, True):
-        for sk in (False, True):
-            assert np.max(np.abs(oracle.block_mass(Q, K, B, 1, rotate=rotate, sampled_keys=sk) - ref)) < 1e-12
+        for mk in (False, True):
+            assert np.max(np.abs(oracle.block_mass(Q, K, B, 1, rotate=rotate, mean_keys=mk) - ref)) < 1e-12
 
 
 def test_gqa_group_mask_shares_lists_and_reaches_tau():

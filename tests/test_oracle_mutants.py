@@ -33,22 +33,49 @@ def _pool_sum(K, S):
 
 
 def _mass_variant(strict_causal=False, no_scale=False, swap=False):
-    def block_mass(Q, K, B, S, row_chunk=2048):
+    def block_mass(Q, K, B, S, row_chunk=2048, rotate=False, mean_keys=False):
         L, H, d = Q.shape
         g = H // K.shape[1]
         Ns, Nb, r = L // S, L // B, B // S
-        Kbar = oracle.pool_keys(K, S)
         pos = oracle.sampled_positions(L, H, S)
         scale = 1.0 if no_scale else 1.0 / math.sqrt(d)
         M = np.zeros((H, Nb, Nb))
         for h in range(H):
-            s = (Q[pos[h], h, :] @ Kbar[:, h // g, :].T) * scale
+            s = (Q[pos[h], h, :] @ K[pos[h], h // g, :].T) * scale
             i, j = np.arange(Ns)[:, None], np.arange(Ns)[None, :]
             s = np.where((j < i) | ((j == i) & (i == 0)) if strict_causal else (j <= i), s, -np.inf)
             P = np.exp(s - s.max(axis=1, keepdims=True))
             P /= P.sum(axis=1, keepdims=True)
             blk = P.reshape(Nb, r, Nb, r).sum(axis=(1, 3))
             M[h] = blk.T if swap else blk
+        return M
+    return block_mass
+
+
+def _sampled_keys_variant(offset_shift=0, kv_by_q_head=False, mean=False):
+    """block_mass whose sampled-key side (R2) takes the key at the head's offset
+    + offset_shift, or on kv head h instead of h // g, or averages the stride."""
+    orig = _orig["block_mass"]
+
+    def block_mass(Q, K, B, S, row_chunk=2048, rotate=False, mean_keys=False):
+        if mean_keys:
+            return orig(Q, K, B, S, row_chunk=row_chunk, rotate=rotate, mean_keys=True)
+        L, H, d = Q.shape
+        g = H // K.shape[1]
+        Ns, Nb, r = L // S, L // B, B // S
+        pos = oracle.rotated_positions(L, H, S) if rotate else oracle.sampled_positions(L, H, S)
+        Kbar = oracle.pool_keys(K, S)
+        M = np.zeros((H, Nb, Nb))
+        for h in range(H):
+            kv = h if kv_by_q_head else h // g
+            kpos = np.arange(Ns) * S + (pos[h] - np.arange(Ns) * S + offset_shift) % S
+            Kb = Kbar[:, kv, :] if mean else K[kpos, kv, :]
+            s = (Q[pos[h], h, :] @ Kb.T) / math.sqrt(d)
+            i, j = np.arange(Ns)[:, None], np.arange(Ns)[None, :]
+            s = np.where(j <= i, s, -np.inf)
+            P = np.exp(s - s.max(axis=1, keepdims=True))
+            P /= P.sum(axis=1, keepdims=True)
+            M[h] = P.reshape(Nb, r, Nb, r).sum(axis=(1, 3))
         return M
     return block_mass
 
@@ -102,6 +129,8 @@ ALL_PINS = [
     pins.test_top_tau_reaching_tau_exactly_stops,
     lambda: pins.test_tau_one_equals_dense_causal_attention(4, 2, 32, 16),
     pins.test_sparse_attention_equals_masked_sdpa,
+    lambda: pins.test_sampled_keys_take_the_heads_own_offset(False),
+    lambda: pins.test_sampled_keys_take_the_heads_own_offset(True),
 ]
 
 MUTANTS = {
@@ -116,6 +145,10 @@ MUTANTS = {
     "ties go to the higher block": ("sorted_order", _order_ties_high),
     "causal mask dropped in attention": ("sparse_attention_block", _attn_variant(no_causal=True)),
     "GQA head mapped with mod": ("sparse_attention_block", _attn_variant(kv_mod=True)),
+    "sampled key one offset late": ("block_mass", _sampled_keys_variant(offset_shift=1)),
+    "sampled key one offset early": ("block_mass", _sampled_keys_variant(offset_shift=-1)),
+    "sampled key from the q head's index": ("block_mass", _sampled_keys_variant(kv_by_q_head=True)),
+    "sampled key replaced by the stride mean": ("block_mass", _sampled_keys_variant(mean=True)),
 }
 
 

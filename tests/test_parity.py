@@ -156,6 +156,44 @@ def test_arbitrary_masks(rr, B, d):
     assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
 
 
+@pytest.mark.parametrize("B,d", [(128, 128), (64, 128)])
+def test_mask_outside_format_is_reported_and_skipped(rr, B, d):
+    """Rows whose block list breaks the mask format are not computed: a key block
+    above the diagonal (J in (I, Nb), still inside the tensor, so nothing is read
+    out of bounds), entries out of order, a repeated entry, a count of 0 and a
+    count above I+1.  Their output rows are zero and rr_check_status reports
+    RR_EMASK; every other row matches the oracle."""
+    L, H, Hkv = 10 * B, 3, 1
+    Nb = L // B
+    q, k, v = gen.make_qkv(L, H, Hkv, d, gen.IID, 43)
+    Q, K, V = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k), gen.bf16_bits_to_f32(v)
+    count, idx = oracle.full_causal_mask(H, Nb)
+    count, idx = count.copy(), np.where(idx < 0, 0, idx).astype(np.int32)
+    bad = {}
+    idx[0, 3, 1] = 7;               bad[(0, 3)] = "future block"        # [0, 7, 2, 3]: J > I
+    count[0, 5], idx[0, 5, :2] = 2, [4, 2];  bad[(0, 5)] = "descending"
+    count[1, 4], idx[1, 4, :3] = 3, [1, 1, 4]; bad[(1, 4)] = "repeated"
+    count[1, 6] = 0;                bad[(1, 6)] = "empty"
+    count[2, 2] = 5;                bad[(2, 2)] = "count above I+1"
+    count[2, 8], idx[2, 8, :2] = 2, [3, Nb - 1]; bad[(2, 8)] = "last entry above the diagonal"
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    o = rr.sparse_attn(to_dev(q), to_dev(k), to_dev(v), torch.from_numpy(count).cuda(),
+                       torch.from_numpy(idx).cuda(), B, ws=ws)
+    assert rr.check_status(ws) == rr.RR_EMASK
+    og = gpu_o_f32(o)
+    good = [(h, I) for h in range(H) for I in range(Nb) if (h, I) not in bad]
+    O_ref = oracle.sparse_attention(Q, K, V, count, idx, B, rows=good)
+    for (h, I), why in bad.items():
+        assert np.all(og[I * B:(I + 1) * B, h, :] == 0.0), why
+    mx, mean = output_errors(og, O_ref)
+    assert mx <= MAX_ERR and mean <= MEAN_ERR, (mx, mean)
+    # the status word is reset by the next call, which then reports ok
+    c2, i2 = oracle.full_causal_mask(H, Nb)
+    rr.sparse_attn(to_dev(q), to_dev(k), to_dev(v), torch.from_numpy(c2).cuda(),
+                   torch.from_numpy(np.where(i2 < 0, 0, i2).astype(np.int32)).cuda(), B, out=o, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+
+
 @pytest.mark.parametrize("B,d", [(128, 128), (64, 64)])
 @pytest.mark.parametrize("slope", [1.5, -1.5, 6.0])
 def test_running_max_moves(rr, slope, B, d):

@@ -1,7 +1,7 @@
 """Parity of the search's sampling variants (rr_search_variant) against the oracle.
 
-V1 rotates the sampled offset across strides, V2 replaces the stride mean of the
-keys by the key at the head's own sampled position, V3 selects one mask per GQA
+V1 rotates the sampled offset across strides, V2 replaces the key at the head's
+own sampled position by the mean of the stride's keys, V3 selects one mask per GQA
 group from the group's summed block mass; any combination.  The per-head block
 mass must agree with the oracle's within the same bound as the plain search, the
 mask within the near-threshold band, and every head of a GQA group must carry
@@ -19,8 +19,8 @@ pytestmark = pytest.mark.gpu
 
 MASS_ERR = 2e-5
 
-ROT, SK, GQA = 1, 2, 4
-ALL_FLAGS = [0, ROT, SK, ROT | SK, GQA, ROT | GQA, SK | GQA, ROT | SK | GQA]
+ROT, MK, GQA = 1, 2, 4
+ALL_FLAGS = [0, ROT, MK, ROT | MK, GQA, ROT | GQA, MK | GQA, ROT | MK | GQA]
 
 
 @pytest.fixture(scope="module")
@@ -49,14 +49,14 @@ def run_case(rr, L, H, Hkv, d, B, S, tau, flags, structure, seed):
     torch.cuda.synchronize()
     count, idx = count.cpu().numpy(), idx.cpu().numpy()
     M_g = mass.cpu().numpy().astype(np.float64)
-    rot, sk, gqa = bool(flags & ROT), bool(flags & SK), bool(flags & GQA)
+    rot, mk, gqa = bool(flags & ROT), bool(flags & MK), bool(flags & GQA)
 
     check_mask_format(count, idx)
-    M_o = oracle.block_mass(Q, K, B, S, rotate=rot, sampled_keys=sk)
+    M_o = oracle.block_mass(Q, K, B, S, rotate=rot, mean_keys=mk)
     tri = np.tri(Nb, dtype=bool)[None]
     err = float(np.max(np.abs(np.where(tri, oracle.normalise_mass(M_g) - oracle.normalise_mass(M_o), 0.0))))
     assert err <= MASS_ERR, f"per-head block mass error {err} (flags {flags})"
-    count_o, idx_o, m_o = oracle.rr_search(Q, K, B, S, tau, rotate=rot, sampled_keys=sk, gqa_mask=gqa)
+    count_o, idx_o, m_o = oracle.rr_search(Q, K, B, S, tau, rotate=rot, mean_keys=mk, gqa_mask=gqa)
     st = compare_masks(count, idx, count_o, idx_o, m_o, tau)
     assert st["blocks_fail"] == 0, (flags, st)
     if gqa:
@@ -82,18 +82,19 @@ def test_variant_flags(rr, flags):
     (512, 3, 3, 64, 64, 64, 0.5, gen.IID),           # r = 1
 ])
 def test_variants_shapes(rr, L, H, Hkv, d, B, S, tau, structure):
-    for flags in (ROT | SK, ROT | SK | GQA, SK):
+    for flags in (ROT, ROT | GQA, MK, ROT | MK | GQA):
         run_case(rr, L, H, Hkv, d, B, S, tau, flags, structure, seed=22)
 
 
 def test_variants_reduce_to_plain_search_at_stride_one(rr):
-    """At S = 1 every query is sampled and each stride is one key: rotation and
-    sampled keys change nothing, so the masks equal the plain search's."""
+    """At S = 1 every query and key is sampled and each stride is one key:
+    rotation and stride-mean keys change nothing, so the masks equal the plain
+    search's."""
     L, H, Hkv, d, B = 1024, 4, 2, 64, 64
     q, k, _ = gen.make_qkv(L, H, Hkv, d, gen.PLANTED, 23)
     qd, kd = to_dev(q), to_dev(k)
     c0, i0 = rr.search(qd, kd, B, 1, 0.9)
-    c1, i1 = rr.search_variant(qd, kd, B, 1, 0.9, ROT | SK)
+    c1, i1 = rr.search_variant(qd, kd, B, 1, 0.9, ROT | MK)
     torch.cuda.synchronize()
     assert torch.equal(c0, c1)
     Nb = L // B
@@ -159,11 +160,11 @@ def test_gqa_mask_long_rows_radix_path(rr):
 
 
 @pytest.mark.slow
-def test_sampled_keys_video64k_full_size(rr):
-    """Sampled keys (and the GQA mask on top) on the full video workload
-    (H=28/Hkv=4, L=65536): masks against the oracle's in full."""
+def test_variants_video64k_full_size(rr):
+    """Stride-mean keys and the GQA mask on the full video workload (H=28/Hkv=4,
+    L=65536): masks against the oracle's in full."""
     cfg = gen.CONFIGS["video64k"]
-    for flags in (SK, SK | GQA):
+    for flags in (MK, GQA):
         count, idx, st = run_case(rr, cfg.L, cfg.H, cfg.Hkv, cfg.d, cfg.B, cfg.S, cfg.tau, flags,
                                   cfg.structure, seed=cfg.seed)
         Nb = cfg.L // cfg.B
