@@ -57,6 +57,19 @@ def block_flops(cfg: gen.Config, visited_blocks: int) -> float:
     return 4.0 * cfg.B * cfg.B * cfg.d * visited_blocks
 
 
+def search_bytes(cfg: gen.Config, visited_blocks: int) -> dict:
+    """Algorithmic HBM bytes of one search stage (sampled keys): every sampled
+    query row and sampled key read once, the lower-triangle block masses
+    written by the score kernel and read by Top-tau, count and idx written."""
+    Ns, Nb = cfg.L // cfg.S, cfg.L // cfg.B
+    rows = Ns * cfg.H * cfg.d * 2
+    tri = cfg.H * Nb * (Nb + 1) // 2 * 4
+    parts = {"q_sampled": rows, "k_sampled": rows, "mass_write": tri, "mass_read": tri,
+             "count_write": cfg.H * Nb * 4, "idx_write": visited_blocks * 4}
+    parts["total"] = sum(parts.values())
+    return parts
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -85,6 +98,20 @@ def kernel_traffic_bytes():
         return float(vals["traffic_bytes_per_launch_full"])
     except (KeyError, ValueError):
         return None
+
+
+def single_thread_tiny_s() -> float:
+    """The oracle (search + attention) on the tiny config with one BLAS thread."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+    cfg = gen.CONFIGS["tiny"]
+    q, k, v = gen.make_config(cfg)
+    Q, K, V = (gen.bf16_bits_to_f32(x) for x in (q, k, v))
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        c, i, _ = oracle.rr_search(Q, K, cfg.B, cfg.S, cfg.tau)
+        oracle.sparse_attention(Q, K, V, c, i, cfg.B)
+        return time.perf_counter() - t0
 
 
 def blas_threads() -> int:
@@ -150,22 +177,29 @@ def oracle_sample(cfg: gen.Config, tau: float, q, k, v, heads=1, rows_per_head=1
 
 def run_reference(args, cfg, tau, world):
     q, k, v = gen.make_config(cfg)
-    times = []
+    measured, extrapolated, rates = [], [], []
     res = None
     for it in range(args.warmup + args.steps):
         res = oracle_sample(cfg, tau, q, k, v, heads=args.ref_heads, rows_per_head=args.ref_rows, seed=it)
         if it >= args.warmup:
-            times.append(res["step_s"])
-    step_s = statistics.mean(times)
-    flops_per_step = res["value"] * 1e12 * res["step_s"]   # extrapolated work of one full step
-    value = flops_per_step / step_s / 1e12
+            measured.append(res["measured_s"])
+            extrapolated.append(res["step_s"])
+            rates.append(res["value"])
+    # a reference step is one bounded sample of the workload: ms_per_step is the
+    # time such a step took; the rate (TFLOP/s over visited blocks) is the
+    # sample's, extrapolated to the layer's work, and the time a whole layer
+    # would take at that rate is reported beside it, not as a step
+    value = statistics.mean(rates)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(measured) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(cfg, tau),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"], "kind": "oracle",
-                         "sample": res["sample"] + "; each step is one such sample"},
+        "extrapolated_full_layer_ms": statistics.mean(extrapolated) * 1e3,
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"], "nproc": os.cpu_count(),
+                         "kind": "oracle",
+                         "sample": res["sample"] + "; each step is one such sample (ms_per_step is its measured "
+                                                   "time; the whole layer is not run)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -307,6 +341,7 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
     # power-capped clock drifts over a run); the speedup compares those two.
     dense_ms = None
     speedup = None
+    alt_reading = None
     if not args.no_dense:
         cd, idd = rr.empty_mask(H, Nb, dev)
         rr.search(qd, kd, B, S, 1.0, count=cd, idx=idd, ws=ws)
@@ -321,15 +356,40 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
             torch.cuda.synchronize(dev)
             return e0.elapsed_time(e1)
 
-        sp, de = [], []
+        # the alternative reading of the key side (stride-mean keys): its mask,
+        # search time and attention time, in the same interleaving
+        ws_mk = rr.workspace(L, H, Hkv, d, B, S, dev, flags=rr.VAR_MEAN_KEYS)
+        cm, im = rr.empty_mask(H, Nb, dev)
+        rr.search_variant(qd, kd, B, S, tau, rr.VAR_MEAN_KEYS, cm, im, ws=ws_mk)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            rr.search_variant(qd, kd, B, S, tau, rr.VAR_MEAN_KEYS, cm, im, ws=ws_mk)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        mk_search_ms = e0.elapsed_time(e1) / 3
+        if rr.check_status(ws_mk) != rr.RR_OK:
+            raise RuntimeError("device-side status of the stride-mean search")
+
+        sp, de, mk = [], [], []
         for _ in range(2):
             sp.append(one(count, idx))
             de.append(one(cd, idd))
+            mk.append(one(cm, im))
         dense_ms = statistics.mean(de)
         speedup = dense_ms / (search_ms + statistics.mean(sp))
         dense_blocks = H * Nb * (Nb + 1) // 2
         dense_tflops = block_flops(cfg, dense_blocks) / (dense_ms / 1e3) / 1e12
-        del cd, idd
+        mk_visited = int(cm.sum().item())
+        alt_reading = {"mean_keys": {
+            "what": "key side of a stride = mean of its S keys (rr_search_variant RR_VAR_MEAN_KEYS)",
+            "search_ms": mk_search_ms, "attn_ms": statistics.mean(mk),
+            "visited_fraction": mk_visited / dense_blocks,
+            "speedup_vs_dense": dense_ms / (mk_search_ms + statistics.mean(mk))},
+            "sampled_keys_default": {"search_ms": search_ms, "attn_ms_interleaved": statistics.mean(sp),
+                                     "visited_fraction": visited / dense_blocks, "speedup_vs_dense": speedup}}
+        del cd, idd, cm, im, ws_mk
 
     # end to end through the public API with host buffers: rr_attention_host
     # copies q, k, v in and o out (page-locked host memory) inside the call,
@@ -362,6 +422,13 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
     peaks = measured_peaks()
     peak = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
     achieved = flops / (attn_ms / 1e3) / 1e12
+    sb = search_bytes(cfg, visited)
+    search_hbm = {"bytes": sb["total"], "gbs": sb["total"] / (search_ms / 1e3) / 1e9,
+                  "frac_of_hbm": sb["total"] / (search_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                  "peak_gbs": peaks["hbm_gbs"], "parts": sb,
+                  "note": "algorithmic bytes of the whole search stage (sampled q rows and keys read once, "
+                          "block-mass write and read, count/idx write) over its CUDA-event time; the stage "
+                          "is bound by tensor and exp work, not by HBM"}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": kernel_traffic_bytes(), "kernel": "bsfa_kernel<128,128>",
                 "peak_kind": f"bf16 dense, sustained ({peaks['source']})"}
@@ -370,6 +437,9 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res = oracle_sample(cfg, tau, q, k, v, heads=args.ref_heads, rows_per_head=args.ref_rows)
         cpu = {k2: res[k2] for k2 in ("value", "unit", "cores", "kind", "sample")}
+        cpu.update({"nproc": os.cpu_count(), "cores_are": "BLAS threads the oracle ran with",
+                    "single_thread_tiny_s": single_thread_tiny_s(),
+                    "measured_sample_s": res["measured_s"]})
 
     if rank == 0:
         line = {
@@ -378,6 +448,7 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator, planted structure)",
             "config": workload_config(cfg, tau),
             "search_ms": search_ms, "attn_ms": attn_ms, "search_share": search_ms / (search_ms + attn_ms),
+            "search_hbm": search_hbm, "alternative_reading": alt_reading,
             "dense_attn_ms": dense_ms, "dense_attn_tflops": dense_tflops if dense_ms else None,
             "speedup_vs_dense": speedup,
             "visited_blocks": visited, "visited_fraction": visited / (H * Nb * (Nb + 1) / 2),

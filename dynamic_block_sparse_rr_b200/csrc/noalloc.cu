@@ -10,38 +10,29 @@
 // holds until the process exits.
 //
 // The entry point itself allocates nothing: it calls no cudaMalloc, cudaFree or
-// allocating library routine.  It resolves the array's device address once per
-// device (cudaGetSymbolAddress, with that device current) and then runs the same
-// kernels as rr_search, with the workspace carved out of the array.
+// allocating library routine.  On every call it asks the runtime for the
+// array's device address on the current device (cudaGetSymbolAddress, a lookup
+// that allocates nothing) and then runs the same kernels as rr_search, with the
+// workspace carved out of the array.  The address is not kept between calls, so
+// a context that was reset in the meantime (cudaDeviceReset) gets the new one.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "rr.h"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = 32ull << 20;   // 32 MiB, see rr.h
-constexpr int kMaxDevices = 64;
 
 // The scratch.  In host code this name is only a stand-in for the symbol, not a
 // device address: it must never be passed to a kernel directly.
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the scratch on the current device (resolved on first use).
+// Device address of the scratch in the current device's context.  The first
+// call in a context also loads this library's device code there.
 rr_status scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RR_ECUDA;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return RR_ECUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return RR_ECUDA;
+  *out = p;
   return RR_OK;
 }
 

@@ -2,6 +2,7 @@
 // workspace carving and stream-ordered launches.  No device memory is
 // allocated here; every buffer is the caller's.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include <vector>
@@ -12,6 +13,15 @@
 namespace {
 
 uint64_t g_wait_limit_ns = 2000000000ull;
+
+// An NVTX range around the host-side enqueue of one stage (visible in a
+// timeline tool next to the kernels it launched; a no-op without one).
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
 
 constexpr size_t kAlign = 256;
 
@@ -165,6 +175,7 @@ rr_status rr_search_variant(const void* q, const void* k, int L, int H, int Hkv,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   unsigned int* status = reinterpret_cast<unsigned int*>(ws + w.status);
   const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
+  const Range range("rr_search");
   if (cudaMemsetAsync(status, 0, sizeof(unsigned int), s) != cudaSuccess) return RR_ECUDA;
   return enqueue_search(q, k, L, H, Hkv, d, B, S, tau, flags, 0, count, idx, mass, ws, w, g, s);
 }
@@ -189,6 +200,7 @@ rr_status rr_sparse_attn(const void* q, const void* k, const void* v, int L, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned int* status = static_cast<unsigned int*>(workspace);
   const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
+  const Range range("rr_sparse_attn");
   if (cudaMemsetAsync(status, 0, sizeof(unsigned int), s) != cudaSuccess) return RR_ECUDA;
   if (rr::launch_bsfa(q, k, v, count, idx, o, L, H, Hkv, d, B, g, s) != cudaSuccess) return RR_ECUDA;
   return RR_OK;
@@ -207,6 +219,7 @@ rr_status rr_attention(const void* q, const void* k, const void* v, int L, int H
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned int* status = static_cast<unsigned int*>(workspace);
   const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
+  const Range range("rr_attention: sparse attention");
   if (rr::launch_bsfa(q, k, v, count, idx, o, L, H, Hkv, d, B, g, s) != cudaSuccess) return RR_ECUDA;
   return RR_OK;
 }
@@ -304,6 +317,7 @@ rr_status rr_attention_host(const void* q_host, const void* k_host, const void* 
     const size_t w = static_cast<size_t>(it.gn) * d * 2;
     int32_t* cc = count + static_cast<size_t>(h_first) * Nb;
     int32_t* ic = idx + static_cast<size_t>(h_first) * Nb * Nb;
+    const Range range("rr_attention_host: item");
     ok = cudaStreamWaitEvent(s, ev_qk[slot], 0) == cudaSuccess;
     if (ok) {
       ok = enqueue_search(base + hl.q, base + hl.k, L, it.gn, 1, d, B, S, tau, 0u, h_first, cc, ic, nullptr,

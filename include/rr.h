@@ -201,9 +201,11 @@ uint64_t rr_set_wait_limit_ns(uint64_t ns);
  *   whose rr_workspace_size exceeds 32 MiB are rejected with RR_ESCRATCH before
  *   anything is enqueued (e.g. H=32, Hkv=8, d=128, B=128, S=16 fits up to
  *   L=32768; L=65536 and beyond do not).
- *   Allocation: none (no cudaMalloc, cudaFree or allocating library call).  The
- *   first call on each device resolves the array's device address with that
- *   device current; make that first call before any stream capture.
+ *   Allocation: none (no cudaMalloc, cudaFree or allocating library call).  Each
+ *   call looks up the array's device address on the current device
+ *   (cudaGetSymbolAddress); the first call in a context also loads the
+ *   library's device code there, so make that first call before any stream
+ *   capture.  Nothing is cached between calls, so a device reset is harmless.
  *   Sharing: every call, on every stream, uses the same array and the array
  *   keeps the last call's contents; calls that overlap on the GPU race, so
  *   serialise them (one stream, or events).
