@@ -50,6 +50,22 @@ V1-V3 Alternatives the pages leave open (off by default): V1 rotates the
     group, selecting on the summed block mass of the group's heads.
                                                               [parity unpinned
     beyond the invariants in tests/test_oracle.py]
+D1-D5 Decode stage.  The TL;DR names decoding-stage sparsification only as a
+    future extension, so every definition here is a reading that carries the
+    prefill rules over to one new token per step.  The query at position t
+    (cache keys 0..t, its own key included):
+    D1  head h scores the keys at its own sampled positions p(h, j) =
+        j*S + (h mod S) that lie at or before t (R1-R2 on the key side);
+    D2  s_j = q . K[p(h,j), h/g] / sqrt(d), softmax over those j;
+    D3  block mass M[J] = sum of P_j over the strides j of block J, J <= J_t =
+        floor(t/B) (a block with no sampled key at or before t has mass 0);
+    D4  Top-tau over J <= J_t as R6, and the current block J_t is always kept
+        (the prefill rule R7 keeps the whole last query block dense; carried
+        over literally it would make every decode step dense, so the decode
+        reading keeps only the block that holds the query and the newest keys);
+    D5  the query attends, with scale 1/sqrt(d), to every key k <= t in the
+        selected blocks.                                       [parity unpinned
+    against the paper: the pages do not describe decoding]
 R9  Mask comparison band (tolerance of the operator's specification): a block
     is near-threshold when the running sum just before or just after it, in
     the R6 order, lies within `band` of tau; a near-tie is a pair of blocks at
@@ -292,3 +308,86 @@ def band_blocks(m_row: np.ndarray, I: int, tau: float, band: float = 1e-4, tie: 
             if t >= k and abs(vals[t] - cut_in) < tie:
                 ties.add(int(order[t]))
     return near, ties
+
+
+# ------------------------------------------------------ D1-D5 decode stage
+def decode_positions(t: int, h: int, S: int) -> np.ndarray:
+    """Sampled key positions of head h for a query at position t (D1):
+    j*S + (h mod S) for every stride j whose sampled position is <= t."""
+    off = h % S
+    if t < off:
+        return np.zeros(0, dtype=np.int64)
+    return np.arange((t - off) // S + 1, dtype=np.int64) * S + off
+
+
+def decode_block_mass(q: np.ndarray, K: np.ndarray, t: int, B: int, S: int) -> np.ndarray:
+    """Block mass of one decode query (D1-D3).  q: [H, d] (the query at position
+    t), K: [L, Hkv, d] with L > t.  Returns [H, J_t + 1] float64, each row
+    summing to 1 (or all zero when the head samples no key at or before t)."""
+    H, d = q.shape
+    g = H // K.shape[1]
+    Jt = t // B
+    M = np.zeros((H, Jt + 1), dtype=np.float64)
+    for h in range(H):
+        pos = decode_positions(t, h, S)
+        if pos.size == 0:
+            continue
+        s = (K[pos, h // g, :].astype(np.float64) @ q[h].astype(np.float64)) / math.sqrt(d)   # D2
+        P = np.exp(s - s.max())
+        P = P / P.sum()
+        np.add.at(M[h], pos // B, P)                                                         # D3
+    return M
+
+
+def decode_select(m_row: np.ndarray, Jt: int, tau: float) -> np.ndarray:
+    """Selected key blocks of one decode query, ascending (D4): the R6 prefix over
+    J <= Jt by (mass desc, J asc), plus the current block Jt."""
+    n = Jt + 1
+    if tau >= 1.0:
+        return np.arange(n, dtype=np.int32)
+    m = m_row[:n]
+    if m.sum() > 0:
+        order = sorted_order(m)
+        run = np.cumsum(m[order] / m.sum())
+        hit = np.nonzero(run >= tau)[0]
+        k = int(hit[0]) + 1 if hit.size else n
+        sel = set(int(j) for j in order[:k])
+    else:
+        sel = set()
+    sel.add(Jt)
+    return np.array(sorted(sel), dtype=np.int32)
+
+
+def decode_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, t: int, blocks, B: int) -> np.ndarray:
+    """Output of one decode query over the listed key blocks (D5).  Returns [H, d]
+    float64; `blocks` is a list (one array of block indices per head)."""
+    H, d = q.shape
+    g = H // K.shape[1]
+    out = np.zeros((H, d), dtype=np.float64)
+    for h in range(H):
+        b = np.asarray(blocks[h], dtype=np.int64)
+        keys = (b[:, None] * B + np.arange(B)[None, :]).reshape(-1)
+        keys = keys[keys <= t]
+        s = (K[keys, h // g, :].astype(np.float64) @ q[h].astype(np.float64)) / math.sqrt(d)
+        p = np.exp(s - s.max())
+        p = p / p.sum()
+        out[h] = p @ V[keys, h // g, :].astype(np.float64)
+    return out
+
+
+def rr_decode(q: np.ndarray, K: np.ndarray, V: np.ndarray, t: int, B: int, S: int, tau: float):
+    """One decode step of one sequence (D1-D5): returns (count [H], idx list per
+    head, normalised mass [H, J_t + 1], output [H, d])."""
+    M = decode_block_mass(q, K, t, B, S)
+    Jt = t // B
+    sel = [decode_select(M[h], Jt, tau) for h in range(q.shape[0])]
+    count = np.array([x.size for x in sel], dtype=np.int32)
+    return count, sel, M, decode_attention(q, K, V, t, sel, B)
+
+
+def decode_band_blocks(m_row: np.ndarray, Jt: int, tau: float, band: float = 1e-4, tie: float = 1e-6):
+    """R9 for a decode row: the blocks whose selection may legitimately differ."""
+    m = np.asarray(m_row[:Jt + 1], dtype=np.float64)
+    tot = m.sum()
+    return band_blocks(m / tot if tot > 0 else m, Jt, tau, band, tie)
+
