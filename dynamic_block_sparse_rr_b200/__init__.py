@@ -24,7 +24,7 @@ RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT, RR_ESCRATCH
 EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status",
            "rr_set_wait_limit_ns", "rr_status_string", "rr_search_static", "rr_mask_recall",
            "rr_workspace_size_variant", "rr_search_variant", "rr_mask_to_dense",
-           "rr_workspace_size_host", "rr_attention_host")
+           "rr_workspace_size_host", "rr_attention_host", "rr_decode_workspace_size", "rr_decode")
 
 # sampling-variant flags of rr_search_variant (rr.h)
 VAR_ROTATE, VAR_MEAN_KEYS, VAR_GQA_MASK = 1, 2, 4
@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
         L.rr_attention_host.argtypes = [vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp, vp, sz, vp, vp]
         L.rr_attention_host.restype = ctypes.c_int
         L.rr_mask_to_dense.restype = ctypes.c_int
+        L.rr_decode_workspace_size.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(sz)]
+        L.rr_decode_workspace_size.restype = ctypes.c_int
+        L.rr_decode.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, vp, sz, vp]
+        L.rr_decode.restype = ctypes.c_int
         L.rr_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.rr_set_wait_limit_ns.restype = ctypes.c_uint64
         L.rr_status_string.argtypes = [i]
@@ -274,3 +278,38 @@ def attention_host(qh, kh, vh, B: int, S: int, tau: float, out=None, count=None,
                                    count.data_ptr(), idx.data_ptr(), out.data_ptr(), ws.data_ptr(), ws.numel(),
                                    s.cuda_stream, copy_stream.cuda_stream), "rr_attention_host")
     return out, count, idx
+
+
+def decode_workspace_size(N: int, Lmax: int, H: int, Hkv: int, d: int, B: int, S: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().rr_decode_workspace_size(N, Lmax, H, Hkv, d, B, S, ctypes.byref(n)), "rr_decode_workspace_size")
+    return n.value
+
+
+def decode(q, k_cache, v_cache, lens, B: int, S: int, tau: float, out=None, count=None, idx=None, ws=None,
+           stream=None):
+    """One decode step: q [N, H, d], caches [N, Lmax, Hkv, d] bf16, lens [N] int32
+    (device) -> (o [N, H, d], count [N, H], idx [N, H, Lmax/B])."""
+    if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("q must be [N, H, d], k_cache and v_cache [N, Lmax, Hkv, d]")
+    N, H, d = q.shape
+    _, Lmax, Hkv, dk = k_cache.shape
+    if k_cache.shape[0] != N or dk != d or lens.shape != (N,) or lens.dtype != torch.int32:
+        raise ValueError("shapes disagree (q, caches, lens)")
+    for t in (q, k_cache, v_cache):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q and the caches must be contiguous bf16 CUDA tensors")
+    Nb = Lmax // B
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if count is None or idx is None:
+        count = torch.empty((N, H), dtype=torch.int32, device=dev)
+        idx = torch.empty((N, H, Nb), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = torch.empty(decode_workspace_size(N, Lmax, H, Hkv, d, B, S), dtype=torch.uint8, device=dev)
+    _check(lib().rr_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), lens.data_ptr(), N, Lmax, H, Hkv,
+                           d, B, S, float(tau), count.data_ptr(), idx.data_ptr(), out.data_ptr(), ws.data_ptr(),
+                           ws.numel(), _stream(stream)), "rr_decode")
+    return out, count, idx
+

@@ -17,7 +17,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "librr.so")
-SOURCES = ["rr_abi.cu", "pool.cu", "search.cu", "topk.cu", "bsfa.cu", "noalloc.cu", "recall.cu", "variants.cu"]
+SOURCES = ["rr_abi.cu", "pool.cu", "search.cu", "topk.cu", "bsfa.cu", "noalloc.cu", "recall.cu", "variants.cu",
+           "decode.cu"]
 HEADERS = ["sm100.cuh", "tmap.h", "rr_internal.h"]
 
 NVCC = os.environ.get("NVCC", "nvcc")

@@ -1,0 +1,508 @@
+// decode.cu — decode-stage sparsification: one new token per sequence attends
+// to its KV cache through a round-robin sampled search and block-sparse
+// attention.  The RRAttention pages name decoding-stage sparsification only as
+// a future extension (sciencestack page, TL;DR); the operator here carries the
+// prefill rules over to a single query at position t = len - 1:
+//   * head h scores the cached keys at its own sampled positions
+//     j*S + (h mod S) <= t, softmax over them, block mass per key block;
+//   * Top-tau over the key blocks J <= t/B as in prefill, and the block that
+//     holds the query (the newest keys) is always kept;
+//   * the query attends to every key <= t of the kept blocks.
+//
+// The path is bound by HBM (the sampled keys, then the kept K and V blocks), so
+// the arithmetic runs on the CUDA cores and the kernels are sized for bytes in
+// flight:
+//   decode_search_kernel   one CTA per (sequence, head): 16-byte loads of the
+//                          sampled key rows, scores to the workspace, block
+//                          mass in shared memory, Top-tau by bisection over the
+//                          mass bits with block-wide sums of fixed-point units
+//                          (the prefill rule), list and a bitmap of the kept
+//                          blocks out;
+//   decode_attn_kernel     one CTA per (sequence, kv head, 32 key blocks): a
+//                          kept block's K and V tiles come in once by TMA
+//                          (two-stage ring) for every query head of the GQA
+//                          group that kept it; per head an online softmax, and
+//                          the chunk's partial (max, sum, output) out;
+//   decode_combine_kernel  one CTA per (sequence, head): the partials merged.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "rr_internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace rr {
+namespace {
+
+constexpr int kDecThreads = 256;
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kMaxPer = (kMaxBlocks + kDecThreads - 1) / kDecThreads;   // masses per thread
+
+// Block-wide sums and max over the 256 threads (fixed order: warp trees, then
+// warp 0 over the warp results).  `buf` holds kDecWarps slots; every thread
+// gets the result.
+template <typename T>
+__device__ __forceinline__ T block_sum(T v, T* buf) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) buf[warp] = v;
+  __syncthreads();
+  T s = buf[0];
+#pragma unroll
+  for (int w = 1; w < kDecWarps; ++w) s += buf[w];
+  return s;
+}
+
+__device__ __forceinline__ float block_max(float v, float* buf) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) buf[warp] = v;
+  __syncthreads();
+  float s = buf[0];
+#pragma unroll
+  for (int w = 1; w < kDecWarps; ++w) s = fmaxf(s, buf[w]);
+  return s;
+}
+
+// Exclusive scan of one u32 per thread in thread order; *total gets the sum.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* buf, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) buf[warp] = x;
+  __syncthreads();
+  uint32_t before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kDecWarps; ++w) {
+    before += w < warp ? buf[w] : 0u;
+    all += buf[w];
+  }
+  *total = all;
+  return before + x - v;
+}
+
+struct DecSearchShared {
+  float q[128];
+  float mass[kMaxBlocks];
+  double dbuf[kDecWarps];
+  float fbuf[kDecWarps];
+  uint32_t ubuf[kDecWarps];
+  uint32_t bits[kMaxBlocks / 32];
+};
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads) decode_search_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const int32_t* __restrict__ lens,
+    int Lmax, int H, int Hkv, int B, int S, float sl2, float tau, float* __restrict__ scores, int Ns_max,
+    int32_t* __restrict__ count, int32_t* __restrict__ idx, uint32_t* __restrict__ bits, int Nbm, int W,
+    unsigned int* status) {
+  __shared__ DecSearchShared sh;
+  const int tid = threadIdx.x;
+  const int n = static_cast<int>(blockIdx.x) / H, h = static_cast<int>(blockIdx.x) % H;
+  const int kvh = h / (H / Hkv);
+  const long long row = static_cast<long long>(n) * H + h;
+  int32_t* out = idx + row * Nbm;
+  uint32_t* obits = bits + row * W;
+  const int len = __ldg(lens + n);
+  if (len < 1 || len > Lmax) {   // not a cache length this call can serve: nothing selected
+    if (tid == 0) {
+      count[row] = 0;
+      atomicCAS(status, 0u, kStatusLenCode | (static_cast<unsigned>(n < (1 << 24) ? n : (1 << 24) - 1) << 8));
+    }
+    for (int w = tid; w < W; w += kDecThreads) obits[w] = 0u;
+    return;
+  }
+  const int t = len - 1, Jt = t / B, nb = Jt + 1, off = h % S, r = B / S;
+  const int ns = t >= off ? (t - off) / S + 1 : 0;   // sampled keys at or before t
+  for (int c = tid; c < D; c += kDecThreads) sh.q[c] = __bfloat162float(q[row * D + c]) * sl2;
+  __syncthreads();
+
+  // scores (log2 units) of the sampled keys, to the workspace row
+  float* sc = scores + row * Ns_max;
+  float lmax = -INFINITY;
+  for (int j = tid; j < ns; j += kDecThreads) {
+    const uint4* kr = reinterpret_cast<const uint4*>(
+        k + ((static_cast<long long>(n) * Lmax + static_cast<long long>(j) * S + off) * Hkv + kvh) * D);
+    uint4 v[D / 8];
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) v[c] = __ldg(kr + c);
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v[c]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(p2[e]);
+        acc0 = fmaf(f.x, sh.q[c * 8 + 2 * e], acc0);
+        acc1 = fmaf(f.y, sh.q[c * 8 + 2 * e + 1], acc1);
+      }
+    }
+    const float s = acc0 + acc1;
+    sc[j] = s;
+    lmax = fmaxf(lmax, s);
+  }
+  const float mx = block_max(lmax, sh.fbuf);
+  __syncthreads();   // the scores of other threads are visible (global writes, same block)
+  // block mass: exp2 of the scores summed over the r strides of each block
+  for (int J = tid; J < nb; J += kDecThreads) {
+    float m = 0.f;
+    const int j1 = min((J + 1) * r, ns);
+    for (int j = J * r; j < j1; ++j) m += exp2f(sc[j] - mx);
+    sh.mass[J] = m;
+  }
+  for (int w = tid; w < (nb + 31) / 32; w += kDecThreads) sh.bits[w] = 0u;
+  __syncthreads();
+
+  // Top-tau over J <= Jt: this thread's contiguous chunk of the row
+  const int per = (nb + kDecThreads - 1) / kDecThreads;
+  const int c0 = min(tid * per, nb), c1 = min(c0 + per, nb);
+  uint32_t key[kMaxPer];
+  double local = 0.0;
+#pragma unroll
+  for (int e = 0; e < kMaxPer; ++e) {
+    key[e] = 0u;
+    if (c0 + e < c1) {
+      const float v = sh.mass[c0 + e];
+      key[e] = __float_as_uint(v);
+      local += static_cast<double>(v);
+    }
+  }
+  uint32_t sel_bits = 0;
+  if (tau < 1.0f) {
+    const double total = block_sum<double>(local, sh.dbuf);
+    const double scale = total > 0.0 ? 2147483648.0 / total : 0.0;
+    auto units = [&](uint32_t kk) { return __double2uint_rn(static_cast<double>(__uint_as_float(kk)) * scale); };
+    uint32_t un[kMaxPer], lsum = 0;
+#pragma unroll
+    for (int e = 0; e < kMaxPer; ++e) {
+      un[e] = c0 + e < c1 ? units(key[e]) : 0u;
+      lsum += un[e];
+    }
+    const uint32_t total_i = block_sum<uint32_t>(lsum, sh.ubuf);
+    if (total_i != 0) {
+      const uint32_t target = static_cast<uint32_t>(
+          fmin(ceil(static_cast<double>(tau) * static_cast<double>(total_i)), static_cast<double>(total_i)));
+      // the largest mass T whose masses at or above it still reach the target
+      uint32_t P = 0;
+      for (int b = 30; b >= 0; --b) {
+        const uint32_t cand = P | (1u << b);
+        uint32_t sge = 0;
+#pragma unroll
+        for (int e = 0; e < kMaxPer; ++e) sge += key[e] >= cand ? un[e] : 0u;
+        if (block_sum<uint32_t>(sge, sh.ubuf) >= target) P = cand;
+      }
+      const uint32_t T = P;
+      uint32_t sgt = 0, my_eq = 0;
+#pragma unroll
+      for (int e = 0; e < kMaxPer; ++e) {
+        sgt += key[e] > T ? un[e] : 0u;
+        my_eq += (c0 + e < c1 && key[e] == T) ? 1u : 0u;
+      }
+      const uint32_t sum_gt = block_sum<uint32_t>(sgt, sh.ubuf);
+      const uint32_t t_val = units(T);
+      const uint32_t k_eq = t_val > 0 ? (target - sum_gt + t_val - 1) / t_val : 1u;
+      uint32_t tot_eq;
+      uint32_t rank = block_excl_scan(my_eq, sh.ubuf, &tot_eq);   // masses equal to T: lowest J first
+#pragma unroll
+      for (int e = 0; e < kMaxPer; ++e) {
+        if (c0 + e < c1) {
+          bool s = key[e] > T;
+          if (key[e] == T) s = rank++ < k_eq;
+          if (s) sel_bits |= 1u << e;
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kMaxPer; ++e)
+      if (c0 + e < c1) sel_bits |= 1u << e;
+  }
+  if (Jt >= c0 && Jt < c1) sel_bits |= 1u << (Jt - c0);   // the block holding the query
+  uint32_t my_sel = __popc(sel_bits), cnt;
+  uint32_t pos = block_excl_scan(my_sel, sh.ubuf, &cnt);
+#pragma unroll
+  for (int e = 0; e < kMaxPer; ++e) {
+    if (sel_bits & (1u << e)) {
+      out[pos++] = c0 + e;
+      atomicOr(&sh.bits[(c0 + e) >> 5], 1u << ((c0 + e) & 31));
+    }
+  }
+  __syncthreads();
+  for (int w = tid; w < W; w += kDecThreads) obits[w] = w < (nb + 31) / 32 ? sh.bits[w] : 0u;
+  if (tid == 0) count[row] = static_cast<int32_t>(cnt);
+}
+
+// ------------------------------------------------------------------ attention
+constexpr int kDecChunk = 32;   // key blocks per attention CTA (one bitmap word per head)
+constexpr int kDecStages = 2;
+
+template <int BN, int D>
+struct DecAttnCfg {
+  static constexpr int kTileBytes = BN * D * 2;
+  static constexpr int kStageBytes = 2 * kTileBytes;   // K and V
+  static constexpr int kSmem = kDecStages * kStageBytes + 1024;
+};
+
+struct DecAttnCtrl {
+  uint64_t full[kDecStages];
+  int abort;
+  uint32_t hbits[8];
+  float q[8][128];
+  float p[8][128];
+};
+
+// Position of the (i+1)-th set bit of `set` (i < popcount).
+__device__ __forceinline__ int nth_bit(uint32_t set, int i) {
+  for (int k = 0; k < i; ++k) set &= set - 1u;
+  return __ffs(static_cast<int>(set)) - 1;
+}
+
+// Byte offset of element (row, c) in a TMA tile of rows x D bf16 stored as D/64
+// column blocks of rows x 128 bytes with the 128-byte swizzle.
+template <int BN>
+__device__ __forceinline__ uint32_t swz(int row, int c) {
+  return static_cast<uint32_t>((c >> 6) * (BN * 128) + row * 128 + ((((c & 63) >> 3) ^ (row & 7)) << 4) + (c & 7) * 2);
+}
+
+template <int BN, int D>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
+    const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lens, const uint32_t* __restrict__ bits,
+    int Lmax, int H, int Hkv, int W, float sl2, float* __restrict__ part, unsigned int* status, uint64_t limit_ns) {
+  using C = DecAttnCfg<BN, D>;
+  constexpr int kKeysPerWarp = BN / kDecWarps;        // 16 (B = 128) or 8 (B = 64)
+  constexpr int kLanesPerKey = 32 / kKeysPerWarp;     // 2 or 4
+  constexpr int kElems = D / kLanesPerKey;            // elements of a key row per lane
+  constexpr int kColsPerLane = D / 32;                // output columns per lane
+  __shared__ DecAttnCtrl ctl;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = static_cast<int>(blockIdx.x), kvh = static_cast<int>(blockIdx.y), n = static_cast<int>(blockIdx.z);
+  const int g = H / Hkv;
+  const int len = __ldg(lens + n);
+  const int t = len - 1;
+  const bool live = len >= 1 && len <= Lmax && chunk * kDecChunk <= t / BN;
+  if (tid < g) ctl.hbits[tid] = live ? __ldg(bits + (static_cast<long long>(n) * H + kvh * g + tid) * W + chunk) : 0u;
+  if (tid == 0) {
+    for (int s = 0; s < kDecStages; ++s) mbar_init(smem_u32(&ctl.full[s]), 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  for (int i = tid; i < g * D; i += kDecThreads) {
+    const int hh = i / D, c = i % D;
+    ctl.q[hh][c] = __bfloat162float(q[(static_cast<long long>(n) * H + kvh * g + hh) * D + c]) * sl2;
+  }
+  __syncthreads();
+  uint32_t any = 0;
+  for (int hh = 0; hh < g; ++hh) any |= ctl.hbits[hh];
+  const Guard guard{&ctl.abort, status, limit_ns};
+
+  // the chunk's kept blocks, ascending; block i of the sequence goes to stage i % 2
+  auto issue = [&](int i, uint32_t set) {
+    const int J = chunk * kDecChunk + nth_bit(set, i);
+    const int st = i % kDecStages;
+    const uint32_t fb = smem_u32(&ctl.full[st]);
+    mbar_expect_tx(fb, C::kStageBytes);
+    uint8_t* dst = smem + st * C::kStageBytes;
+    const int r0 = n * Lmax + J * BN;
+    for (int a = 0; a < D / 64; ++a) {
+      tma_load_3d(smem_u32(dst + a * BN * 128), &mk, fb, a * 64, kvh, r0);
+      tma_load_3d(smem_u32(dst + C::kTileBytes + a * BN * 128), &mv, fb, a * 64, kvh, r0);
+    }
+  };
+  const int n_blk = __popc(any);
+  int issued = 0;   // thread 0: copies issued so far
+  if (tid == 0) {
+    tma_prefetch_desc(&mk);
+    tma_prefetch_desc(&mv);
+    for (; issued < n_blk && issued < kDecStages; ++issued) issue(issued, any);
+  }
+
+  // per head (warp w < g): running max m, sum l and the lane's output columns
+  float m_run = -INFINITY, l_run = 0.f, o_acc[kColsPerLane];
+#pragma unroll
+  for (int c = 0; c < kColsPerLane; ++c) o_acc[c] = 0.f;
+  const int key = warp * kKeysPerWarp + lane / kLanesPerKey;   // S phase: this lane's key
+  const int part_e = (lane % kLanesPerKey) * kElems;            // and its share of d
+  bool ok = true;
+  for (int i = 0; i < n_blk; ++i) {
+    const int J = chunk * kDecChunk + nth_bit(any, i);
+    const uint32_t jb = 1u << (J - chunk * kDecChunk);
+    const int st = i % kDecStages;
+    if (!wait_bar(smem_u32(&ctl.full[st]), (i / kDecStages) & 1, guard, 1)) ok = false;
+    if (!__syncthreads_and(ok)) break;
+    const uint8_t* ks = smem + st * C::kStageBytes;
+    const uint8_t* vs = ks + C::kTileBytes;
+    // S phase: the lane's part of its key row, dotted with each head that kept J
+    {
+      float kf[kElems];
+#pragma unroll
+      for (int c = 0; c < kElems; c += 8) {
+        const uint4 v4 = *reinterpret_cast<const uint4*>(ks + swz<BN>(key, part_e + c));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(p2[e]);
+          kf[c + 2 * e] = f.x;
+          kf[c + 2 * e + 1] = f.y;
+        }
+      }
+      const bool masked = J * BN + key > t;
+      for (int hh = 0; hh < g; ++hh) {
+        if (!(ctl.hbits[hh] & jb)) continue;   // uniform across the CTA
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < kElems; c += 2) {
+          a0 = fmaf(kf[c], ctl.q[hh][part_e + c], a0);
+          a1 = fmaf(kf[c + 1], ctl.q[hh][part_e + c + 1], a1);
+        }
+        float s = a0 + a1;
+#pragma unroll
+        for (int x = 1; x < kLanesPerKey; x <<= 1) s += __shfl_xor_sync(0xffffffffu, s, x);
+        if (lane % kLanesPerKey == 0) ctl.p[hh][key] = masked ? -INFINITY : s;
+      }
+    }
+    __syncthreads();
+    // softmax and P V: warp w serves head w
+    if (warp < g && (ctl.hbits[warp] & jb)) {
+      float s[BN / 32];
+      float bm = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < BN / 32; ++e) {
+        s[e] = ctl.p[warp][lane + 32 * e];
+        bm = fmaxf(bm, s[e]);
+      }
+#pragma unroll
+      for (int x = 16; x > 0; x >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, x));
+      const float m_new = fmaxf(m_run, bm);   // finite: key J*B <= t, since J <= t/B
+      const float alpha = exp2f(m_run - m_new);
+      float ps = 0.f;
+#pragma unroll
+      for (int e = 0; e < BN / 32; ++e) {
+        const float p = exp2f(s[e] - m_new);
+        ps += p;
+        ctl.p[warp][lane + 32 * e] = p;
+      }
+#pragma unroll
+      for (int x = 16; x > 0; x >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, x);
+      l_run = l_run * alpha + ps;
+      m_run = m_new;
+#pragma unroll
+      for (int c = 0; c < kColsPerLane; ++c) o_acc[c] *= alpha;
+      __syncwarp();
+      const int c0 = lane * kColsPerLane;
+#pragma unroll 4
+      for (int kk = 0; kk < BN; ++kk) {
+        const float p = ctl.p[warp][kk];
+        if constexpr (kColsPerLane == 4) {
+          const uint2 v2 = *reinterpret_cast<const uint2*>(vs + swz<BN>(kk, c0));
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v2);
+          const float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
+          o_acc[0] = fmaf(p, f0.x, o_acc[0]);
+          o_acc[1] = fmaf(p, f0.y, o_acc[1]);
+          o_acc[2] = fmaf(p, f1.x, o_acc[2]);
+          o_acc[3] = fmaf(p, f1.y, o_acc[3]);
+        } else {
+          const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(vs + swz<BN>(kk, c0));
+          const float2 f = __bfloat1622float2(v2);
+          o_acc[0] = fmaf(p, f.x, o_acc[0]);
+          o_acc[1] = fmaf(p, f.y, o_acc[1]);
+        }
+      }
+    }
+    __syncthreads();   // stage st is free again
+    if (tid == 0 && issued < n_blk) issue(issued++, any);
+  }
+  // in-flight copies land before the CTA exits (only after an abort can any be left)
+  if (tid == 0) {
+    for (int i = (issued > kDecStages ? issued - kDecStages : 0); i < issued; ++i)
+      drain_bar(smem_u32(&ctl.full[i % kDecStages]), (i / kDecStages) & 1, kDrainLimitNs);
+  }
+  // partial of each head of the group for this chunk: (max, sum, output columns)
+  if (warp < g) {
+    const long long prow = ((static_cast<long long>(n) * H + kvh * g + warp) * W + chunk) * (D + 2);
+    const bool has = ok && live && (ctl.hbits[warp] != 0u);
+    if (lane == 0) {
+      part[prow] = has ? m_run : -INFINITY;
+      part[prow + 1] = has ? l_run : 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < kColsPerLane; ++c) part[prow + 2 + lane * kColsPerLane + c] = has ? o_acc[c] : 0.f;
+  }
+}
+
+// Partials of the chunks of one (sequence, head) merged: O = sum_c o_c 2^(m_c - M)
+// / sum_c l_c 2^(m_c - M), M the largest m_c.  One thread per output column.
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ part, const int32_t* __restrict__ lens,
+                                                          int Lmax, int B, int W, __nv_bfloat16* __restrict__ o) {
+  const int n = static_cast<int>(blockIdx.y);
+  const long long row = static_cast<long long>(n) * gridDim.x + blockIdx.x;   // n * H + h
+  const int c = threadIdx.x;
+  const int len = __ldg(lens + n);
+  const int nc = (len >= 1 && len <= Lmax) ? ((len - 1) / B) / kDecChunk + 1 : 0;
+  const float* p = part + row * W * (D + 2);
+  float M = -INFINITY;
+  for (int k = 0; k < nc; ++k) M = fmaxf(M, p[k * (D + 2)]);
+  float L = 0.f, O = 0.f;
+  if (M > -INFINITY) {
+    for (int k = 0; k < nc; ++k) {
+      const float mk = p[k * (D + 2)];
+      if (mk == -INFINITY) continue;
+      const float f = exp2f(mk - M);
+      L += p[k * (D + 2) + 1] * f;
+      O += p[k * (D + 2) + 2 + c] * f;
+    }
+  }
+  o[row * D + c] = __float2bfloat16(L > 0.f ? O / L : 0.f);
+}
+
+template <int BN, int D>
+cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const int32_t* lens, int N, int Lmax, int H,
+                            int Hkv, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                            const DecodeScratch& w, const DeviceGuardArgs& g, cudaStream_t stream) {
+  const int Nbm = Lmax / BN, W = (Nbm + 31) / 32;
+  const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+  decode_search_kernel<D><<<static_cast<unsigned>(N) * H, kDecThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), lens, Lmax, H, Hkv, BN, S, sl2, tau,
+      w.scores, Lmax / S, count, idx, w.bits, Nbm, W, g.status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap mk, mv;
+  const uint64_t rows = static_cast<uint64_t>(N) * Lmax;
+  if (!make_tmap_rows(&mk, k, rows, Hkv, D, BN) || !make_tmap_rows(&mv, v, rows, Hkv, D, BN))
+    return cudaErrorInvalidValue;
+  using C = DecAttnCfg<BN, D>;
+  static std::atomic<uint64_t> smem_set{0};
+  if ((e = set_smem_limit_once(decode_attn_kernel<BN, D>, C::kSmem, smem_set)) != cudaSuccess) return e;
+  decode_attn_kernel<BN, D><<<dim3(W, Hkv, N), kDecThreads, C::kSmem, stream>>>(
+      mk, mv, static_cast<const __nv_bfloat16*>(q), lens, w.bits, Lmax, H, Hkv, W, sl2, w.part, g.status, g.limit_ns);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  decode_combine_kernel<D><<<dim3(H, N), D, 0, stream>>>(w.part, lens, Lmax, BN, W, static_cast<__nv_bfloat16*>(o));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const int32_t* lens, int N, int Lmax, int H,
+                          int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                          const DecodeScratch& w, const DeviceGuardArgs& g, cudaStream_t stream) {
+  if (B == 128 && d == 128) return launch_decode_t<128, 128>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, count, idx, o, w, g, stream);
+  if (B == 128 && d == 64) return launch_decode_t<128, 64>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, count, idx, o, w, g, stream);
+  if (B == 64 && d == 128) return launch_decode_t<64, 128>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, count, idx, o, w, g, stream);
+  if (B == 64 && d == 64) return launch_decode_t<64, 64>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, count, idx, o, w, g, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rr

@@ -132,6 +132,37 @@ HostLayout carve_host(int L, int H, int Hkv, int d, int B, int S) {
   return w;
 }
 
+// Decode workspace: the status word, the sampled scores [N, H, Lmax/S] fp32, the
+// kept-block bitmaps [N, H, W] u32 and the attention partials [N, H, W, d+2]
+// fp32, W = ceil(Lmax/B / 32).
+struct DecodeLayout {
+  size_t status, scores, bits, part, total;
+};
+
+DecodeLayout carve_decode(int N, int Lmax, int H, int d, int B, int S) {
+  DecodeLayout w;
+  const size_t rows = static_cast<size_t>(N) * H;
+  const size_t W = (static_cast<size_t>(Lmax / B) + 31) / 32;
+  size_t off = kAlign;
+  w.status = 0;
+  w.scores = off; off += round_up(rows * (Lmax / S) * 4);
+  w.bits = off; off += round_up(rows * W * 4);
+  w.part = off; off += round_up(rows * W * (d + 2) * 4);
+  w.total = off;
+  return w;
+}
+
+rr_status check_decode_shape(int N, int Lmax, int H, int Hkv, int d, int B, int S) {
+  if (N <= 0 || Lmax <= 0 || H <= 0 || Hkv <= 0 || S <= 0) return RR_EINVAL;
+  if (H % Hkv != 0 || B <= 0 || B % S != 0 || Lmax % B != 0) return RR_EINVAL;
+  if (d != 64 && d != 128) return RR_EUNSUPPORTED;
+  if (B != 64 && B != 128) return RR_EUNSUPPORTED;
+  if (H / Hkv > 8) return RR_EUNSUPPORTED;
+  if (Lmax / B > rr::kMaxBlocks) return RR_EUNSUPPORTED;
+  if (static_cast<long long>(N) * Lmax >= (1ll << 31)) return RR_EUNSUPPORTED;
+  return RR_OK;
+}
+
 rr_status check_ws(void* ws, size_t ws_bytes, const Layout& w) {
   if (!ws) return RR_EINVAL;
   if (reinterpret_cast<uintptr_t>(ws) % kAlign) return RR_EALIGN;
@@ -337,6 +368,41 @@ rr_status rr_attention_host(const void* q_host, const void* k_host, const void* 
   return ok ? RR_OK : RR_ECUDA;
 }
 
+rr_status rr_decode_workspace_size(int N, int Lmax, int H, int Hkv, int d, int B, int S, size_t* bytes) {
+  if (!bytes) return RR_EINVAL;
+  const rr_status st = check_decode_shape(N, Lmax, H, Hkv, d, B, S);
+  if (st != RR_OK) return st;
+  *bytes = carve_decode(N, Lmax, H, d, B, S).total;
+  return RR_OK;
+}
+
+rr_status rr_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int N, int Lmax,
+                    int H, int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  rr_status st = check_decode_shape(N, Lmax, H, Hkv, d, B, S);
+  if (st != RR_OK) return st;
+  if (!(tau > 0.0f) || tau != tau) return RR_EINVAL;
+  if (!q || !k_cache || !v_cache || !lens || !count || !idx || !o || !workspace) return RR_EINVAL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(count) ||
+      !aligned16(idx) || (reinterpret_cast<uintptr_t>(lens) & 3u))
+    return RR_EALIGN;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return RR_EALIGN;
+  const DecodeLayout w = carve_decode(N, Lmax, H, d, B, S);
+  if (workspace_bytes < w.total) return RR_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned int* status = reinterpret_cast<unsigned int*>(ws + w.status);
+  const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
+  const rr::DecodeScratch sc{reinterpret_cast<float*>(ws + w.scores), reinterpret_cast<uint32_t*>(ws + w.bits),
+                             reinterpret_cast<float*>(ws + w.part)};
+  const Range range("rr_decode");
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned int), s) != cudaSuccess) return RR_ECUDA;
+  if (rr::launch_decode(q, k_cache, v_cache, lens, N, Lmax, H, Hkv, d, B, S, tau, count, idx, o, sc, g, s) !=
+      cudaSuccess)
+    return RR_ECUDA;
+  return RR_OK;
+}
+
 rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int Nb, uint8_t* dense, void* stream) {
   if (!count || !idx || !dense || H <= 0 || Nb <= 0) return RR_EINVAL;
   if (Nb > rr::kMaxBlocks) return RR_EUNSUPPORTED;
@@ -354,6 +420,7 @@ rr_status rr_check_status(void* workspace, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return RR_ECUDA;
   if ((host & 0xFFu) == rr::kStatusTimeoutCode) return RR_ETIMEOUT;
   if ((host & 0xFFu) == rr::kStatusMaskCode) return RR_EMASK;
+  if ((host & 0xFFu) == rr::kStatusLenCode) return RR_EINVAL;
   return host == 0 ? RR_OK : RR_ECUDA;
 }
 

@@ -86,6 +86,25 @@ constexpr unsigned kStatusTimeoutCode = 5u;
 // list outside the mask format (bits 8..31: the row h*Nb + I, saturated).
 constexpr unsigned kStatusMaskCode = 7u;
 
+// Low byte of the workspace status word when a decode call met a cache length
+// outside [1, Lmax] (bits 8..31: the sequence, saturated).
+constexpr unsigned kStatusLenCode = 8u;
+
+// Decode-stage scratch (workspace regions): sampled scores [N, H, Lmax/S] fp32,
+// kept-block bitmaps [N, H, W] u32 (W = ceil(Lmax/B / 32)), and the attention
+// partials [N, H, W, d + 2] fp32 (max, sum, output columns per 32-block chunk).
+struct DecodeScratch {
+  float* scores;
+  uint32_t* bits;
+  float* part;
+};
+
+// Decode stage: search, block-sparse attention and combine for one new token per
+// sequence.  q, o: [N, H, d]; k, v: [N, Lmax, Hkv, d]; lens: [N] cache lengths.
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const int32_t* lens, int N, int Lmax, int H,
+                          int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                          const DecodeScratch& w, const DeviceGuardArgs& g, cudaStream_t stream);
+
 // Largest Nb = L/B the kernels accept (bounded by the on-chip list / sort buffers).
 constexpr int kMaxBlocks = 4096;
 

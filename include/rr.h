@@ -182,9 +182,44 @@ rr_status rr_mask_recall(const float* mass, const int32_t* count, const int32_t*
 rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int Nb, uint8_t* dense,
                            void* stream);
 
+/* Decode stage: one new token per sequence, over its KV cache.  The pages name
+ * decoding-stage sparsification only as a future extension (sciencestack page,
+ * TL;DR); this call carries the prefill rules over to the query at position
+ * t = lens[n] - 1 of each sequence n:
+ *   Search:   head h scores the cached keys at its own sampled positions
+ *             j*S + (h mod S) <= t (the prefill sampling on the key side):
+ *             s_j = q . k_j / sqrt(d), softmax over those j, mass of key block
+ *             J = sum over its strides, for J <= t/B.
+ *   Top-tau:  as rr_search (mass desc, J asc, shortest prefix with share >= tau,
+ *             fixed-point sums); the block t/B, which holds the query and the
+ *             newest keys, is always kept.  (Prefill keeps the whole last query
+ *             block dense; carried over literally that would make every decode
+ *             step dense.)
+ *   Attention: the query attends, with scale 1/sqrt(d), to every key <= t of
+ *             the kept blocks; fp32 softmax and accumulation, bf16 output.
+ * In:  q [N,H,d] bf16 (the new tokens' queries); k_cache, v_cache [N,Lmax,Hkv,d]
+ *      bf16 with the new tokens' keys and values already written at position
+ *      lens[n]-1; lens [N] int32 (device), each in [1, Lmax].
+ * Out: count [N,H] int32, idx [N,H,Lmax/B] int32 (kept blocks ascending, valid
+ *      below count), o [N,H,d] bf16.  All device memory, caller-owned.
+ * Workspace: rr_decode_workspace_size bytes, 256-byte aligned (sampled scores,
+ * kept-block bitmaps, per-chunk attention partials, status word).
+ * Requires Lmax % B == 0, B % S == 0, d and B in {64, 128}, H/Hkv <= 8,
+ * Lmax/B <= 4096.  A length outside [1, Lmax] is found on the device: that
+ * sequence gets count 0 and a zero output, and rr_check_status returns
+ * RR_EINVAL.  Kernels: a search CTA per (sequence, head), an attention CTA per
+ * (sequence, kv head, 32 key blocks) that loads each kept K/V block once for
+ * every head of its GQA group that kept it, and a combine CTA per
+ * (sequence, head). */
+rr_status rr_decode_workspace_size(int N, int Lmax, int H, int Hkv, int d, int B, int S, size_t* bytes);
+rr_status rr_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int N, int Lmax,
+                    int H, int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, returns the device-side status recorded since the
- * last rr_* call that started on this workspace (RR_OK, RR_ETIMEOUT or
- * RR_EMASK), and RR_ECUDA if the stream reports an error. */
+ * last rr_* call that started on this workspace (RR_OK, RR_ETIMEOUT, RR_EMASK,
+ * or RR_EINVAL for a decode cache length out of range), and RR_ECUDA if the
+ * stream reports an error. */
 rr_status rr_check_status(void* workspace, void* stream);
 
 /* Sets the bound, in nanoseconds, of every device-side wait of later launches

@@ -183,3 +183,33 @@ def test_host_workspace_and_rejections(rr):
     assert call(ws=g + 64) == rr.RR_EALIGN
     assert call(nb=nws - 1) == rr.RR_EINVAL
     assert call(tau=0.0) == rr.RR_EINVAL
+
+
+def test_decode_workspace_and_rejections(rr):
+    lib = rr.lib()
+    g = 1 << 20
+    n = ctypes.c_size_t()
+    N, Lmax, H, Hkv, d, B, S = 2, 4096, 8, 2, 128, 128, 16
+    assert lib.rr_decode_workspace_size(N, Lmax, H, Hkv, d, B, S, ctypes.byref(n)) == rr.RR_OK
+    W = (Lmax // B + 31) // 32
+    # status word, sampled scores, bitmaps and per-chunk partials
+    assert n.value >= N * H * (Lmax // S) * 4 + N * H * W * 4 + N * H * W * (d + 2) * 4
+    nws = n.value
+    for args, code in [((N, Lmax, H, 3, d, B, S), rr.RR_EINVAL),        # H % Hkv
+                       ((N, 4000, H, Hkv, d, B, S), rr.RR_EINVAL),      # Lmax % B
+                       ((N, Lmax, H, Hkv, d, B, 3), rr.RR_EINVAL),      # B % S
+                       ((N, Lmax, 18, 2, d, B, S), rr.RR_EUNSUPPORTED),  # more than 8 heads per kv head
+                       ((N, Lmax, H, Hkv, 96, B, S), rr.RR_EUNSUPPORTED),
+                       ((0, Lmax, H, Hkv, d, B, S), rr.RR_EINVAL)]:
+        assert lib.rr_decode_workspace_size(*args, ctypes.byref(n)) == code, args
+
+    def call(q=g, lens=g, tau=0.9, ws=g, nws=nws):
+        return lib.rr_decode(q, g, g, lens, N, Lmax, H, Hkv, d, B, S, tau, g, g, g, ws, nws, None)
+
+    assert call(q=None) == rr.RR_EINVAL
+    assert call(tau=0.0) == rr.RR_EINVAL
+    assert call(q=g + 8) == rr.RR_EALIGN
+    assert call(lens=g + 2) == rr.RR_EALIGN
+    assert call(ws=g + 16) == rr.RR_EALIGN
+    assert call(nws=nws - 1) == rr.RR_EINVAL
+
