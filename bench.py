@@ -391,6 +391,8 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
                                      "visited_fraction": visited / dense_blocks, "speedup_vs_dense": speedup}}
         del cd, idd, cm, im, ws_mk
 
+    decode = None if args.no_decode else measure_decode(args, rr, cfg, tau, qd, kd, vd, dev, stream)
+
     # end to end through the public API with host buffers: rr_attention_host
     # copies q, k, v in and o out (page-locked host memory) inside the call,
     # pipelined against the kernels item by item
@@ -448,7 +450,7 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator, planted structure)",
             "config": workload_config(cfg, tau),
             "search_ms": search_ms, "attn_ms": attn_ms, "search_share": search_ms / (search_ms + attn_ms),
-            "search_hbm": search_hbm, "alternative_reading": alt_reading,
+            "search_hbm": search_hbm, "alternative_reading": alt_reading, "decode": decode,
             "dense_attn_ms": dense_ms, "dense_attn_tflops": dense_tflops if dense_ms else None,
             "speedup_vs_dense": speedup,
             "visited_blocks": visited, "visited_fraction": visited / (H * Nb * (Nb + 1) / 2),
@@ -459,6 +461,94 @@ def run_ours(args, cfg, tau, rank, world, local_rank):
             "gpu_launches": gpu_launches, "clocks": clk, "roofline": roofline, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+
+
+def decode_bytes(cfg: gen.Config, lens, count, idx) -> dict:
+    """Algorithmic HBM bytes of one decode step: each head's sampled keys up to
+    its query, the union over a kv group's heads of the kept K and V blocks (the
+    attention kernel loads a kept block once per group), q and o."""
+    H, Hkv, d, B, S = cfg.H, cfg.Hkv, cfg.d, cfg.B, cfg.S
+    g = H // Hkv
+    row = d * 2
+    keys = kv = 0
+    for n, ln in enumerate(lens):
+        t = ln - 1
+        for h in range(H):
+            off = h % S
+            keys += ((t - off) // S + 1 if t >= off else 0) * row
+        for c in range(Hkv):
+            union = set()
+            for h in range(c * g, (c + 1) * g):
+                union.update(idx[n, h, :count[n, h]].tolist())
+            for J in union:
+                kv += 2 * (min(B, t + 1 - J * B)) * row
+    qo = 2 * len(lens) * H * row
+    return {"sampled_keys": keys, "kv_blocks": kv, "q_o": qo, "total": keys + kv + qo}
+
+
+def measure_decode(args, rr, cfg, tau, qd, kd, vd, dev, stream):
+    """Decode step of the layer for a batch of sequences: caches are copies of
+    the resident layer's k and v, sequence n holds L - 1000 n keys and its query
+    is the layer's query at its last position.  Times rr_decode (CUDA events)
+    at tau and at tau = 1 (every block kept), interleaved."""
+    import torch
+    Nd = args.decode_batch
+    L, H, Hkv, d, B, S = cfg.L, cfg.H, cfg.Hkv, cfg.d, cfg.B, cfg.S
+    lens = [L - 1000 * n for n in range(Nd)]
+    kc = kd.unsqueeze(0).expand(Nd, -1, -1, -1).contiguous()
+    vc = vd.unsqueeze(0).expand(Nd, -1, -1, -1).contiguous()
+    qq = torch.stack([qd[ln - 1] for ln in lens]).contiguous()
+    ld = torch.tensor(lens, dtype=torch.int32, device=dev)
+    ws = torch.empty(rr.decode_workspace_size(Nd, L, H, Hkv, d, B, S), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(qq)
+    cnt = torch.empty((Nd, H), dtype=torch.int32, device=dev)
+    idx = torch.empty((Nd, H, L // B), dtype=torch.int32, device=dev)
+    cnt1, idx1 = torch.empty_like(cnt), torch.empty_like(idx)
+
+    def timed(t_, c_, i_, reps=10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            rr.decode(qq, kc, vc, ld, B, S, t_, out=out, count=c_, idx=i_, ws=ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    for _ in range(3):
+        timed(tau, cnt, idx, 1)
+        timed(1.0, cnt1, idx1, 1)
+    sp, de = [], []
+    for _ in range(3):
+        sp.append(timed(tau, cnt, idx))
+        de.append(timed(1.0, cnt1, idx1))
+    if rr.check_status(ws) != rr.RR_OK:
+        raise RuntimeError("device-side status of the decode step")
+    ms, dense_ms = statistics.median(sp), statistics.median(de)
+    c_h, i_h = cnt.cpu().numpy(), idx.cpu().numpy()
+    byts = decode_bytes(cfg, lens, c_h, i_h)
+    gbs = byts["total"] / (ms / 1e3) / 1e9
+    peak = measured_peaks()["hbm_gbs"]
+    visited = float(c_h.sum()) / sum(H * ((ln - 1) // B + 1) for ln in lens)
+    del kc, vc, ws
+    torch.cuda.empty_cache()
+    return {"what": "rr_decode: one new token per sequence over its KV cache (search, block-sparse attention, "
+                    "combine); caches are copies of this layer, sequence n holds L - 1000 n keys",
+            "batch": Nd, "us_per_step": ms * 1e3, "dense_us_per_step": dense_ms * 1e3,
+            "speedup_vs_dense": dense_ms / ms, "visited_fraction": visited,
+            "hbm": {"bytes": byts["total"], "gbs": gbs, "frac_of_hbm": gbs / peak, "peak_gbs": peak,
+                    "parts": byts}}
+
+
+def run_decode_only(args, cfg, tau):
+    import torch
+    import dynamic_block_sparse_rr_b200 as rr
+    dev = torch.device("cuda", 0)
+    q, k, v = gen.make_config(cfg)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    del q, k, v
+    res = measure_decode(args, rr, cfg, tau, qd, kd, vd, dev, torch.cuda.current_stream(dev))
+    print(json.dumps({"diagnostic": "decode step", "config": workload_config(cfg, tau), "decode": res}), flush=True)
 
 
 def run_recall(args, cfg, taus, variants=(0,)):
@@ -588,6 +678,10 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=16, help="oracle sample: attention rows per head")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
+    ap.add_argument("--decode-batch", type=int, default=8, help="sequences per decode step")
+    ap.add_argument("--decode", action="store_true",
+                    help="decode-step measurement only (one JSON line), on the chosen config's layer")
     ap.add_argument("--recall", action="store_true",
                     help="mask diagnostics instead of timing: recall of exact attention mass per tau")
     ap.add_argument("--sweep", action="store_true",
@@ -612,6 +706,10 @@ def main():
     if args.sweep:
         if rank == 0:
             run_sweep(args)
+        return
+    if args.decode:
+        if rank == 0:
+            run_decode_only(args, cfg, tau)
         return
     if args.recall:
         if rank == 0:

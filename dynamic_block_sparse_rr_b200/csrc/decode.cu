@@ -9,20 +9,24 @@
 //     holds the query (the newest keys) is always kept;
 //   * the query attends to every key <= t of the kept blocks.
 //
-// The path is bound by HBM (the sampled keys, then the kept K and V blocks), so
-// the arithmetic runs on the CUDA cores and the kernels are sized for bytes in
-// flight:
+// The path is bound by HBM (the sampled keys, then the kept K and V blocks); the
+// kernels are sized for bytes in flight and kept lean in instructions:
 //   decode_search_kernel   one CTA per (sequence, head): 16-byte loads of the
 //                          sampled key rows, scores to the workspace, block
 //                          mass in shared memory, Top-tau by bisection over the
 //                          mass bits with block-wide sums of fixed-point units
 //                          (the prefill rule), list and a bitmap of the kept
 //                          blocks out;
-//   decode_attn_kernel     one CTA per (sequence, kv head, 32 key blocks): a
+//   decode_attn_kernel     one CTA per (sequence, kv head, 16 key blocks): a
 //                          kept block's K and V tiles come in once by TMA
-//                          (two-stage ring) for every query head of the GQA
-//                          group that kept it; per head an online softmax, and
-//                          the chunk's partial (max, sum, output) out;
+//                          (three-stage ring) for every query head of the GQA
+//                          group that kept it.  The group's <= 8 heads are the 8
+//                          columns of m16n8k16 tensor-core tiles (mma.sync), so
+//                          the two small contractions per block (scores of 128
+//                          keys, P V) are a few instructions per warp; each warp
+//                          keeps an online softmax over its 16 keys of every
+//                          block, and the warps' partials merge into the
+//                          chunk's partial (max, sum, output);
 //   decode_combine_kernel  one CTA per (sequence, head): the partials merged.
 #include <cuda_bf16.h>
 #include <math.h>
@@ -242,22 +246,23 @@ __global__ void __launch_bounds__(kDecThreads) decode_search_kernel(
 }
 
 // ------------------------------------------------------------------ attention
-constexpr int kDecChunk = 32;   // key blocks per attention CTA (one bitmap word per head)
-constexpr int kDecStages = 2;
+constexpr int kDecChunk = 16;   // key blocks per attention CTA (half a bitmap word)
+constexpr int kDecStages = 3;
 
 template <int BN, int D>
 struct DecAttnCfg {
   static constexpr int kTileBytes = BN * D * 2;
   static constexpr int kStageBytes = 2 * kTileBytes;   // K and V
   static constexpr int kSmem = kDecStages * kStageBytes + 1024;
+  static_assert(kDecWarps * 8 * D * 4 <= kStageBytes, "the warp partials fit in one stage");
 };
 
 struct DecAttnCtrl {
   uint64_t full[kDecStages];
   int abort;
   uint32_t hbits[8];
-  float q[8][128];
-  float p[8][128];
+  float2 ml[kDecWarps][8];                 // warp partials: (max, sum) per head
+  __nv_bfloat16 p[kDecWarps][8][24];       // per warp: P of its 16 keys, [head][key] (rows padded)
 };
 
 // Position of the (i+1)-th set bit of `set` (i < popcount).
@@ -267,50 +272,95 @@ __device__ __forceinline__ int nth_bit(uint32_t set, int i) {
 }
 
 // Byte offset of element (row, c) in a TMA tile of rows x D bf16 stored as D/64
-// column blocks of rows x 128 bytes with the 128-byte swizzle.
+// column blocks of rows x 128 bytes with the 128-byte swizzle (c a multiple of 8
+// when used as a 16-byte row address).
 template <int BN>
 __device__ __forceinline__ uint32_t swz(int row, int c) {
   return static_cast<uint32_t>((c >> 6) * (BN * 128) + row * 128 + ((((c & 63) >> 3) ^ (row & 7)) << 4) + (c & 7) * 2);
 }
 
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col).
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One CTA per (sequence n, kv head, 16 key blocks).  Each kept block J comes in
+// once for the whole GQA group; the group's heads are the 8 columns of
+// m16n8k16 tiles (heads beyond the group and heads that did not keep J are
+// masked).  Warp w owns keys 16w..16w+15 of every block and keeps its own
+// online softmax and O^T over them (a split over keys inside the CTA):
+//   S^T [16 keys x heads] = K_J [16 keys x d] . Q^T [d x heads]
+//   per head: running max and sum over the warp's keys, P (bf16) re-laid from
+//   the accumulator fragment to the operand fragment through a small per-warp
+//   buffer
+//   O^T [d x heads] += V_J^T [d x 16 keys] . P^T [16 keys x heads]
+// No cross-warp exchange per block: one barrier frees the stage.  At the end the
+// eight warp partials are merged into the chunk's partial.  Q^T stays in
+// registers as B fragments; K comes in as A fragments by ldmatrix, V^T by
+// ldmatrix.trans, both from the 128-byte swizzled TMA tiles.
 template <int BN, int D>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
     const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lens, const uint32_t* __restrict__ bits,
-    int Lmax, int H, int Hkv, int W, float sl2, float* __restrict__ part, unsigned int* status, uint64_t limit_ns) {
+    int Lmax, int H, int Hkv, int W, int NC, float sl2, float* __restrict__ part, unsigned int* status,
+    uint64_t limit_ns) {
   using C = DecAttnCfg<BN, D>;
-  constexpr int kKeysPerWarp = BN / kDecWarps;        // 16 (B = 128) or 8 (B = 64)
-  constexpr int kLanesPerKey = 32 / kKeysPerWarp;     // 2 or 4
-  constexpr int kElems = D / kLanesPerKey;            // elements of a key row per lane
-  constexpr int kColsPerLane = D / 32;                // output columns per lane
+  constexpr int kKeyWarps = BN / 16;  // warps that own keys (8 at B = 128, 4 at B = 64)
+  constexpr int kDSteps = D / 16;     // k-steps of S (over d)
+  constexpr int kOTiles = D / 16;     // d-row tiles of O^T
   __shared__ DecAttnCtrl ctl;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gid = lane >> 2, tig = lane & 3;   // mma fragment coordinates
   const int chunk = static_cast<int>(blockIdx.x), kvh = static_cast<int>(blockIdx.y), n = static_cast<int>(blockIdx.z);
   const int g = H / Hkv;
   const int len = __ldg(lens + n);
   const int t = len - 1;
-  const bool live = len >= 1 && len <= Lmax && chunk * kDecChunk <= t / BN;
-  if (tid < g) ctl.hbits[tid] = live ? __ldg(bits + (static_cast<long long>(n) * H + kvh * g + tid) * W + chunk) : 0u;
+  const int J0 = chunk * kDecChunk;
+  const bool live = len >= 1 && len <= Lmax && J0 <= t / BN;
+  if (tid < 8) {
+    uint32_t b = 0u;
+    if (live && tid < g) b = __ldg(bits + (static_cast<long long>(n) * H + kvh * g + tid) * W + (J0 >> 5));
+    ctl.hbits[tid] = (b >> (J0 & 31)) & ((1u << kDecChunk) - 1u);
+  }
   if (tid == 0) {
     for (int s = 0; s < kDecStages; ++s) mbar_init(smem_u32(&ctl.full[s]), 1);
     ctl.abort = 0;
     fence_mbar_init();
   }
-  for (int i = tid; i < g * D; i += kDecThreads) {
-    const int hh = i / D, c = i % D;
-    ctl.q[hh][c] = __bfloat162float(q[(static_cast<long long>(n) * H + kvh * g + hh) * D + c]) * sl2;
+  // Q^T as B fragments: b0 = Q[head gid][16 ks + 2 tig, +1], b1 = the same at +8
+  uint32_t qb[kDSteps][2];
+  {
+    const bool hv = gid < g;
+    const __nv_bfloat16* qr = q + (static_cast<long long>(n) * H + kvh * g + (hv ? gid : 0)) * D;
+#pragma unroll
+    for (int ks = 0; ks < kDSteps; ++ks) {
+      qb[ks][0] = hv ? __ldg(reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * tig)) : 0u;
+      qb[ks][1] = hv ? __ldg(reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * tig + 8)) : 0u;
+    }
   }
   __syncthreads();
   uint32_t any = 0;
   for (int hh = 0; hh < g; ++hh) any |= ctl.hbits[hh];
   const Guard guard{&ctl.abort, status, limit_ns};
 
-  // the chunk's kept blocks, ascending; block i of the sequence goes to stage i % 2
-  auto issue = [&](int i, uint32_t set) {
-    const int J = chunk * kDecChunk + nth_bit(set, i);
+  // the chunk's kept blocks, ascending; block i of the sequence goes to stage i % kDecStages
+  auto issue = [&](int i) {
+    const int J = J0 + nth_bit(any, i);
     const int st = i % kDecStages;
     const uint32_t fb = smem_u32(&ctl.full[st]);
     mbar_expect_tx(fb, C::kStageBytes);
@@ -326,119 +376,143 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
   if (tid == 0) {
     tma_prefetch_desc(&mk);
     tma_prefetch_desc(&mv);
-    for (; issued < n_blk && issued < kDecStages; ++issued) issue(issued, any);
+    for (; issued < n_blk && issued < kDecStages; ++issued) issue(issued);
   }
 
-  // per head (warp w < g): running max m, sum l and the lane's output columns
-  float m_run = -INFINITY, l_run = 0.f, o_acc[kColsPerLane];
+  // This warp's running max and sum for the lane's two head columns (2 tig,
+  // 2 tig + 1), and its O^T tiles (d rows 16 mt + gid and + 8, the same columns).
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  float o_acc[kOTiles][4];
 #pragma unroll
-  for (int c = 0; c < kColsPerLane; ++c) o_acc[c] = 0.f;
-  const int key = warp * kKeysPerWarp + lane / kLanesPerKey;   // S phase: this lane's key
-  const int part_e = (lane % kLanesPerKey) * kElems;            // and its share of d
+  for (int mt = 0; mt < kOTiles; ++mt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) o_acc[mt][c] = 0.f;
+  const int mi = lane >> 3, ri = lane & 7;   // ldmatrix: this lane's matrix and row
   bool ok = true;
   for (int i = 0; i < n_blk; ++i) {
-    const int J = chunk * kDecChunk + nth_bit(any, i);
-    const uint32_t jb = 1u << (J - chunk * kDecChunk);
+    const int J = J0 + nth_bit(any, i);
+    const uint32_t jb = 1u << (J - J0);
     const int st = i % kDecStages;
     if (!wait_bar(smem_u32(&ctl.full[st]), (i / kDecStages) & 1, guard, 1)) ok = false;
     if (!__syncthreads_and(ok)) break;
-    const uint8_t* ks = smem + st * C::kStageBytes;
-    const uint8_t* vs = ks + C::kTileBytes;
-    // S phase: the lane's part of its key row, dotted with each head that kept J
-    {
-      float kf[kElems];
+    if (warp < kKeyWarps) {
+      const uint32_t ks_base = smem_u32(smem + st * C::kStageBytes);
+      const uint32_t vs_base = ks_base + C::kTileBytes;
+      const bool keep0 = 2 * tig < g && (ctl.hbits[2 * tig] & jb);
+      const bool keep1 = 2 * tig + 1 < g && (ctl.hbits[2 * tig + 1] & jb);
+      // S^T tile: keys 16w + gid (acc 0, 1) and 16w + gid + 8 (acc 2, 3)
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kElems; c += 8) {
-        const uint4 v4 = *reinterpret_cast<const uint4*>(ks + swz<BN>(key, part_e + c));
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(p2[e]);
-          kf[c + 2 * e] = f.x;
-          kf[c + 2 * e + 1] = f.y;
-        }
+      for (int ks = 0; ks < kDSteps; ++ks) {
+        uint32_t a[4];
+        ldsm_x4(ks_base + swz<BN>(16 * warp + (mi & 1) * 8 + ri, 16 * ks + (mi >> 1) * 8), a);
+        mma_bf16(acc, a, qb[ks][0], qb[ks][1]);
       }
-      const bool masked = J * BN + key > t;
-      for (int hh = 0; hh < g; ++hh) {
-        if (!(ctl.hbits[hh] & jb)) continue;   // uniform across the CTA
-        float a0 = 0.f, a1 = 0.f;
+      const int key0 = J * BN + 16 * warp + gid;
+      const bool v0 = key0 <= t, v1 = key0 + 8 <= t;
+      const float s0 = (keep0 && v0) ? acc[0] * sl2 : -INFINITY;
+      const float s1 = (keep1 && v0) ? acc[1] * sl2 : -INFINITY;
+      const float s2 = (keep0 && v1) ? acc[2] * sl2 : -INFINITY;
+      const float s3 = (keep1 && v1) ? acc[3] * sl2 : -INFINITY;
+      // per head column: max over the warp's 16 keys
+      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
-        for (int c = 0; c < kElems; c += 2) {
-          a0 = fmaf(kf[c], ctl.q[hh][part_e + c], a0);
-          a1 = fmaf(kf[c + 1], ctl.q[hh][part_e + c + 1], a1);
-        }
-        float s = a0 + a1;
-#pragma unroll
-        for (int x = 1; x < kLanesPerKey; x <<= 1) s += __shfl_xor_sync(0xffffffffu, s, x);
-        if (lane % kLanesPerKey == 0) ctl.p[hh][key] = masked ? -INFINITY : s;
+      for (int x = 4; x < 32; x <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, x));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, x));
       }
-    }
-    __syncthreads();
-    // softmax and P V: warp w serves head w
-    if (warp < g && (ctl.hbits[warp] & jb)) {
-      float s[BN / 32];
-      float bm = -INFINITY;
+      const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+      // a column with nothing so far and nothing now keeps alpha 1 (its O is 0)
+      const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m_run[0] - mn0);
+      const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m_run[1] - mn1);
+      const __nv_bfloat16 p0 = __float2bfloat16(s0 == -INFINITY ? 0.f : exp2f(s0 - mn0));
+      const __nv_bfloat16 p1 = __float2bfloat16(s1 == -INFINITY ? 0.f : exp2f(s1 - mn1));
+      const __nv_bfloat16 p2 = __float2bfloat16(s2 == -INFINITY ? 0.f : exp2f(s2 - mn0));
+      const __nv_bfloat16 p3 = __float2bfloat16(s3 == -INFINITY ? 0.f : exp2f(s3 - mn1));
+      // sums of the bf16 P that P V uses
+      float sm0 = __bfloat162float(p0) + __bfloat162float(p2), sm1 = __bfloat162float(p1) + __bfloat162float(p3);
 #pragma unroll
-      for (int e = 0; e < BN / 32; ++e) {
-        s[e] = ctl.p[warp][lane + 32 * e];
-        bm = fmaxf(bm, s[e]);
+      for (int x = 4; x < 32; x <<= 1) {
+        sm0 += __shfl_xor_sync(0xffffffffu, sm0, x);
+        sm1 += __shfl_xor_sync(0xffffffffu, sm1, x);
       }
-#pragma unroll
-      for (int x = 16; x > 0; x >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, x));
-      const float m_new = fmaxf(m_run, bm);   // finite: key J*B <= t, since J <= t/B
-      const float alpha = exp2f(m_run - m_new);
-      float ps = 0.f;
-#pragma unroll
-      for (int e = 0; e < BN / 32; ++e) {
-        const float p = exp2f(s[e] - m_new);
-        ps += p;
-        ctl.p[warp][lane + 32 * e] = p;
-      }
-#pragma unroll
-      for (int x = 16; x > 0; x >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, x);
-      l_run = l_run * alpha + ps;
-      m_run = m_new;
-#pragma unroll
-      for (int c = 0; c < kColsPerLane; ++c) o_acc[c] *= alpha;
+      l_run[0] = l_run[0] * al0 + sm0;
+      l_run[1] = l_run[1] * al1 + sm1;
+      m_run[0] = mn0;
+      m_run[1] = mn1;
+      // P from the accumulator layout (key rows, head columns) to the operand
+      // layout (b0 = P[head gid][keys 2 tig, +1], b1 = keys + 8)
+      __nv_bfloat16(*pw)[24] = ctl.p[warp];
+      pw[2 * tig][gid] = p0;
+      pw[2 * tig + 1][gid] = p1;
+      pw[2 * tig][gid + 8] = p2;
+      pw[2 * tig + 1][gid + 8] = p3;
       __syncwarp();
-      const int c0 = lane * kColsPerLane;
-#pragma unroll 4
-      for (int kk = 0; kk < BN; ++kk) {
-        const float p = ctl.p[warp][kk];
-        if constexpr (kColsPerLane == 4) {
-          const uint2 v2 = *reinterpret_cast<const uint2*>(vs + swz<BN>(kk, c0));
-          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v2);
-          const float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
-          o_acc[0] = fmaf(p, f0.x, o_acc[0]);
-          o_acc[1] = fmaf(p, f0.y, o_acc[1]);
-          o_acc[2] = fmaf(p, f1.x, o_acc[2]);
-          o_acc[3] = fmaf(p, f1.y, o_acc[3]);
-        } else {
-          const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(vs + swz<BN>(kk, c0));
-          const float2 f = __bfloat1622float2(v2);
-          o_acc[0] = fmaf(p, f.x, o_acc[0]);
-          o_acc[1] = fmaf(p, f.y, o_acc[1]);
-        }
+      const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&pw[gid][2 * tig]);
+      const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&pw[gid][2 * tig + 8]);
+      __syncwarp();
+#pragma unroll
+      for (int mt = 0; mt < kOTiles; ++mt) {
+        o_acc[mt][0] *= al0;
+        o_acc[mt][1] *= al1;
+        o_acc[mt][2] *= al0;
+        o_acc[mt][3] *= al1;
+        uint32_t a[4];
+        ldsm_x4_t(vs_base + swz<BN>(16 * warp + (mi >> 1) * 8 + ri, 16 * mt + (mi & 1) * 8), a);
+        mma_bf16(o_acc[mt], a, b0, b1);
       }
     }
     __syncthreads();   // stage st is free again
-    if (tid == 0 && issued < n_blk) issue(issued++, any);
+    if (tid == 0 && issued < n_blk) issue(issued++);
   }
   // in-flight copies land before the CTA exits (only after an abort can any be left)
   if (tid == 0) {
     for (int i = (issued > kDecStages ? issued - kDecStages : 0); i < issued; ++i)
       drain_bar(smem_u32(&ctl.full[i % kDecStages]), (i / kDecStages) & 1, kDrainLimitNs);
   }
-  // partial of each head of the group for this chunk: (max, sum, output columns)
-  if (warp < g) {
-    const long long prow = ((static_cast<long long>(n) * H + kvh * g + warp) * W + chunk) * (D + 2);
-    const bool has = ok && live && (ctl.hbits[warp] != 0u);
-    if (lane == 0) {
-      part[prow] = has ? m_run : -INFINITY;
-      part[prow + 1] = has ? l_run : 0.f;
+  const bool done = __syncthreads_and(ok) && live;
+  // merge the warp partials: stage 0 holds each warp's O^T as [warp][head][d] fp32
+  float* ow = reinterpret_cast<float*>(smem);
+  if (warp < kKeyWarps) {
+    if (gid == 0) {
+      ctl.ml[warp][2 * tig] = make_float2(m_run[0], l_run[0]);
+      ctl.ml[warp][2 * tig + 1] = make_float2(m_run[1], l_run[1]);
     }
 #pragma unroll
-    for (int c = 0; c < kColsPerLane; ++c) part[prow + 2 + lane * kColsPerLane + c] = has ? o_acc[c] : 0.f;
+    for (int mt = 0; mt < kOTiles; ++mt) {
+      const int d0 = 16 * mt + gid;
+      ow[(warp * 8 + 2 * tig) * D + d0] = o_acc[mt][0];
+      ow[(warp * 8 + 2 * tig + 1) * D + d0] = o_acc[mt][1];
+      ow[(warp * 8 + 2 * tig) * D + d0 + 8] = o_acc[mt][2];
+      ow[(warp * 8 + 2 * tig + 1) * D + d0 + 8] = o_acc[mt][3];
+    }
+  }
+  __syncthreads();
+  // thread layout: head hh = tid / 32 (one warp per head), d columns lane, lane + 32, ...
+  const int hh = warp;
+  if (hh < g) {
+    const long long prow = ((static_cast<long long>(n) * H + kvh * g + hh) * NC + chunk) * (D + 2);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kKeyWarps; ++w) M = fmaxf(M, ctl.ml[w][hh].x);
+    const bool has = done && M > -INFINITY;
+    float f[kKeyWarps], L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kKeyWarps; ++w) {
+      const float2 ml = ctl.ml[w][hh];
+      f[w] = (has && ml.x > -INFINITY) ? exp2f(ml.x - M) : 0.f;
+      L += ml.y * f[w];
+    }
+    if (lane == 0) {
+      part[prow] = has ? M : -INFINITY;
+      part[prow + 1] = has ? L : 0.f;
+    }
+    for (int d = lane; d < D; d += 32) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kKeyWarps; ++w) acc += ow[(w * 8 + hh) * D + d] * f[w];
+      part[prow + 2 + d] = has ? acc : 0.f;
+    }
   }
 }
 
@@ -446,13 +520,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
 // / sum_c l_c 2^(m_c - M), M the largest m_c.  One thread per output column.
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ part, const int32_t* __restrict__ lens,
-                                                          int Lmax, int B, int W, __nv_bfloat16* __restrict__ o) {
+                                                          int Lmax, int B, int NC, __nv_bfloat16* __restrict__ o) {
   const int n = static_cast<int>(blockIdx.y);
   const long long row = static_cast<long long>(n) * gridDim.x + blockIdx.x;   // n * H + h
   const int c = threadIdx.x;
   const int len = __ldg(lens + n);
   const int nc = (len >= 1 && len <= Lmax) ? ((len - 1) / B) / kDecChunk + 1 : 0;
-  const float* p = part + row * W * (D + 2);
+  const float* p = part + row * NC * (D + 2);
   float M = -INFINITY;
   for (int k = 0; k < nc; ++k) M = fmaxf(M, p[k * (D + 2)]);
   float L = 0.f, O = 0.f;
@@ -486,10 +560,12 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
   using C = DecAttnCfg<BN, D>;
   static std::atomic<uint64_t> smem_set{0};
   if ((e = set_smem_limit_once(decode_attn_kernel<BN, D>, C::kSmem, smem_set)) != cudaSuccess) return e;
-  decode_attn_kernel<BN, D><<<dim3(W, Hkv, N), kDecThreads, C::kSmem, stream>>>(
-      mk, mv, static_cast<const __nv_bfloat16*>(q), lens, w.bits, Lmax, H, Hkv, W, sl2, w.part, g.status, g.limit_ns);
+  const int NC = (Nbm + kDecChunk - 1) / kDecChunk;
+  decode_attn_kernel<BN, D><<<dim3(NC, Hkv, N), kDecThreads, C::kSmem, stream>>>(
+      mk, mv, static_cast<const __nv_bfloat16*>(q), lens, w.bits, Lmax, H, Hkv, W, NC, sl2, w.part, g.status,
+      g.limit_ns);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  decode_combine_kernel<D><<<dim3(H, N), D, 0, stream>>>(w.part, lens, Lmax, BN, W, static_cast<__nv_bfloat16*>(o));
+  decode_combine_kernel<D><<<dim3(H, N), D, 0, stream>>>(w.part, lens, Lmax, BN, NC, static_cast<__nv_bfloat16*>(o));
   return cudaGetLastError();
 }
 

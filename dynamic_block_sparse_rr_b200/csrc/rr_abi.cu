@@ -133,8 +133,8 @@ HostLayout carve_host(int L, int H, int Hkv, int d, int B, int S) {
 }
 
 // Decode workspace: the status word, the sampled scores [N, H, Lmax/S] fp32, the
-// kept-block bitmaps [N, H, W] u32 and the attention partials [N, H, W, d+2]
-// fp32, W = ceil(Lmax/B / 32).
+// kept-block bitmaps [N, H, W] u32 (W = ceil(Lmax/B / 32)) and the attention
+// partials [N, H, NC, d+2] fp32, one per 16-block chunk (NC = ceil(Lmax/B / 16)).
 struct DecodeLayout {
   size_t status, scores, bits, part, total;
 };
@@ -143,11 +143,12 @@ DecodeLayout carve_decode(int N, int Lmax, int H, int d, int B, int S) {
   DecodeLayout w;
   const size_t rows = static_cast<size_t>(N) * H;
   const size_t W = (static_cast<size_t>(Lmax / B) + 31) / 32;
+  const size_t NC = (static_cast<size_t>(Lmax / B) + 15) / 16;
   size_t off = kAlign;
   w.status = 0;
   w.scores = off; off += round_up(rows * (Lmax / S) * 4);
   w.bits = off; off += round_up(rows * W * 4);
-  w.part = off; off += round_up(rows * W * (d + 2) * 4);
+  w.part = off; off += round_up(rows * NC * (d + 2) * 4);
   w.total = off;
   return w;
 }

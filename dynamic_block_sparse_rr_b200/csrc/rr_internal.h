@@ -92,7 +92,8 @@ constexpr unsigned kStatusLenCode = 8u;
 
 // Decode-stage scratch (workspace regions): sampled scores [N, H, Lmax/S] fp32,
 // kept-block bitmaps [N, H, W] u32 (W = ceil(Lmax/B / 32)), and the attention
-// partials [N, H, W, d + 2] fp32 (max, sum, output columns per 32-block chunk).
+// partials [N, H, NC, d + 2] fp32 (max, sum, output columns per 16-block chunk,
+// NC = ceil(Lmax/B / 16)).
 struct DecodeScratch {
   float* scores;
   uint32_t* bits;

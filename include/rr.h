@@ -208,7 +208,7 @@ rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int 
  * Lmax/B <= 4096.  A length outside [1, Lmax] is found on the device: that
  * sequence gets count 0 and a zero output, and rr_check_status returns
  * RR_EINVAL.  Kernels: a search CTA per (sequence, head), an attention CTA per
- * (sequence, kv head, 32 key blocks) that loads each kept K/V block once for
+ * (sequence, kv head, 16 key blocks) that loads each kept K/V block once for
  * every head of its GQA group that kept it, and a combine CTA per
  * (sequence, head). */
 rr_status rr_decode_workspace_size(int N, int Lmax, int H, int Hkv, int d, int B, int S, size_t* bytes);

@@ -191,9 +191,9 @@ def test_decode_workspace_and_rejections(rr):
     n = ctypes.c_size_t()
     N, Lmax, H, Hkv, d, B, S = 2, 4096, 8, 2, 128, 128, 16
     assert lib.rr_decode_workspace_size(N, Lmax, H, Hkv, d, B, S, ctypes.byref(n)) == rr.RR_OK
-    W = (Lmax // B + 31) // 32
+    W, NC = (Lmax // B + 31) // 32, (Lmax // B + 15) // 16
     # status word, sampled scores, bitmaps and per-chunk partials
-    assert n.value >= N * H * (Lmax // S) * 4 + N * H * W * 4 + N * H * W * (d + 2) * 4
+    assert n.value >= N * H * (Lmax // S) * 4 + N * H * W * 4 + N * H * NC * (d + 2) * 4
     nws = n.value
     for args, code in [((N, Lmax, H, 3, d, B, S), rr.RR_EINVAL),        # H % Hkv
                        ((N, 4000, H, Hkv, d, B, S), rr.RR_EINVAL),      # Lmax % B
