@@ -11,9 +11,11 @@
 //
 // The path is bound by HBM (the sampled keys, then the kept K and V blocks); the
 // kernels are sized for bytes in flight and kept lean in instructions:
-//   decode_search_kernel   one CTA per (sequence, head): 16-byte loads of the
-//                          sampled key rows, scores to the workspace, block
-//                          mass in shared memory, Top-tau by bisection over the
+//   decode_search_kernel   one CTA per (sequence, head): the head's sampled key
+//                          rows come in as 128-row TMA tiles of a zero-copy
+//                          strided view (two-stage ring), scores to the
+//                          workspace, block mass in shared memory, Top-tau by
+//                          bisection over the
 //                          mass bits with block-wide sums of fixed-point units
 //                          (the prefill rule), list and a bitmap of the kept
 //                          blocks out;
@@ -94,8 +96,18 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* buf, u
   return before + x - v;
 }
 
+constexpr int kSearchTile = 128;   // sampled keys per TMA tile of the search
+constexpr int kSearchStages = 2;
+
+// Byte offset of element (row, c) of a 128-row TMA tile (128-byte swizzle, D/64
+// column blocks of 128 rows x 128 bytes); c a multiple of 8.
+__device__ __forceinline__ uint32_t swz128(int row, int c) {
+  return static_cast<uint32_t>((c >> 6) * (128 * 128) + row * 128 + ((((c & 63) >> 3) ^ (row & 7)) << 4));
+}
+
 struct DecSearchShared {
-  float q[128];
+  uint64_t full[kSearchStages];
+  int abort;
   float mass[kMaxBlocks];
   double dbuf[kDecWarps];
   float fbuf[kDecWarps];
@@ -105,11 +117,14 @@ struct DecSearchShared {
 
 template <int D>
 __global__ void __launch_bounds__(kDecThreads) decode_search_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const int32_t* __restrict__ lens,
+    const __grid_constant__ CUtensorMap mks, const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lens,
     int Lmax, int H, int Hkv, int B, int S, float sl2, float tau, float* __restrict__ scores, int Ns_max,
     int32_t* __restrict__ count, int32_t* __restrict__ idx, uint32_t* __restrict__ bits, int Nbm, int W,
-    unsigned int* status) {
+    unsigned int* status, uint64_t limit_ns) {
+  constexpr int kTileBytes = kSearchTile * D * 2;
   __shared__ DecSearchShared sh;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int n = static_cast<int>(blockIdx.x) / H, h = static_cast<int>(blockIdx.x) % H;
   const int kvh = h / (H / Hkv);
@@ -127,32 +142,78 @@ __global__ void __launch_bounds__(kDecThreads) decode_search_kernel(
   }
   const int t = len - 1, Jt = t / B, nb = Jt + 1, off = h % S, r = B / S;
   const int ns = t >= off ? (t - off) / S + 1 : 0;   // sampled keys at or before t
-  for (int c = tid; c < D; c += kDecThreads) sh.q[c] = __bfloat162float(q[row * D + c]) * sl2;
+  const int nt = (ns + kSearchTile - 1) / kSearchTile;
+  if (tid == 0) {
+    for (int st = 0; st < kSearchStages; ++st) mbar_init(smem_u32(&sh.full[st]), 1);
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  // lanes 2k and 2k+1 score key k of a tile, each over half of d; the half of
+  // q they need stays in registers
+  const int kr = tid >> 1, half = tid & 1;
+  float qr[D / 2];
+#pragma unroll
+  for (int c = 0; c < D / 2; c += 2) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + row * D + half * (D / 2) + c));
+    qr[c] = f.x * sl2;
+    qr[c + 1] = f.y * sl2;
+  }
   __syncthreads();
-
+  const Guard guard{&sh.abort, status, limit_ns};
+  // tile i: the sampled keys of strides 128 i .. 128 i + 127 of sequence n
+  auto issue = [&](int i) {
+    const int st = i % kSearchStages;
+    const uint32_t fb = smem_u32(&sh.full[st]);
+    mbar_expect_tx(fb, kTileBytes);
+    uint8_t* dst = smem + st * kTileBytes;
+    for (int a = 0; a < D / 64; ++a)
+      tma_load_4d(smem_u32(dst + a * kSearchTile * 128), &mks, fb, a * 64, kvh, off,
+                  n * (Lmax / S) + i * kSearchTile);
+  };
+  int issued = 0;
+  if (tid == 0) {
+    tma_prefetch_desc(&mks);
+    for (; issued < nt && issued < kSearchStages; ++issued) issue(issued);
+  }
   // scores (log2 units) of the sampled keys, to the workspace row
   float* sc = scores + row * Ns_max;
   float lmax = -INFINITY;
-  for (int j = tid; j < ns; j += kDecThreads) {
-    const uint4* kr = reinterpret_cast<const uint4*>(
-        k + ((static_cast<long long>(n) * Lmax + static_cast<long long>(j) * S + off) * Hkv + kvh) * D);
-    uint4 v[D / 8];
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) v[c] = __ldg(kr + c);
+  bool ok = true;
+  for (int i = 0; i < nt; ++i) {
+    const int st = i % kSearchStages;
+    if (!wait_bar(smem_u32(&sh.full[st]), (i / kSearchStages) & 1, guard, 1)) ok = false;
+    if (!__syncthreads_and(ok)) break;
+    const uint8_t* tile = smem + st * kTileBytes;
     float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v[c]);
+    for (int c = 0; c < D / 2; c += 8) {
+      const uint4 v4 = *reinterpret_cast<const uint4*>(tile + swz128(kr, half * (D / 2) + c));
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 f = __bfloat1622float2(p2[e]);
-        acc0 = fmaf(f.x, sh.q[c * 8 + 2 * e], acc0);
-        acc1 = fmaf(f.y, sh.q[c * 8 + 2 * e + 1], acc1);
+        acc0 = fmaf(f.x, qr[c + 2 * e], acc0);
+        acc1 = fmaf(f.y, qr[c + 2 * e + 1], acc1);
       }
     }
-    const float s = acc0 + acc1;
-    sc[j] = s;
-    lmax = fmaxf(lmax, s);
+    float sv = acc0 + acc1;
+    sv += __shfl_xor_sync(0xffffffffu, sv, 1);
+    const int j = i * kSearchTile + kr;
+    if (j < ns) {
+      if (half == 0) sc[j] = sv;
+      lmax = fmaxf(lmax, sv);
+    }
+    __syncthreads();   // stage st is free again
+    if (tid == 0 && issued < nt) issue(issued++);
+  }
+  if (tid == 0) {
+    for (int i = (issued > kSearchStages ? issued - kSearchStages : 0); i < issued; ++i)
+      drain_bar(smem_u32(&sh.full[i % kSearchStages]), (i / kSearchStages) & 1, kDrainLimitNs);
+  }
+  if (!__syncthreads_and(ok)) {   // a wait ran out (status recorded): nothing selected
+    if (tid == 0) count[row] = 0;
+    for (int w = tid; w < W; w += kDecThreads) obits[w] = 0u;
+    return;
   }
   const float mx = block_max(lmax, sh.fbuf);
   __syncthreads();   // the scores of other threads are visible (global writes, same block)
@@ -548,15 +609,19 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
                             const DecodeScratch& w, const DeviceGuardArgs& g, cudaStream_t stream) {
   const int Nbm = Lmax / BN, W = (Nbm + 31) / 32;
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-  decode_search_kernel<D><<<static_cast<unsigned>(N) * H, kDecThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), lens, Lmax, H, Hkv, BN, S, sl2, tau,
-      w.scores, Lmax / S, count, idx, w.bits, Nbm, W, g.status);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  CUtensorMap mk, mv;
+  CUtensorMap mks, mk, mv;
   const uint64_t rows = static_cast<uint64_t>(N) * Lmax;
-  if (!make_tmap_rows(&mk, k, rows, Hkv, D, BN) || !make_tmap_rows(&mv, v, rows, Hkv, D, BN))
+  if (!make_tmap_sampled(&mks, k, rows, Hkv, D, S, kSearchTile) || !make_tmap_rows(&mk, k, rows, Hkv, D, BN) ||
+      !make_tmap_rows(&mv, v, rows, Hkv, D, BN))
     return cudaErrorInvalidValue;
+  constexpr int kSearchSmem = kSearchStages * kSearchTile * D * 2 + 1024;
+  static std::atomic<uint64_t> search_smem_set{0};
+  cudaError_t e = set_smem_limit_once(decode_search_kernel<D>, kSearchSmem, search_smem_set);
+  if (e != cudaSuccess) return e;
+  decode_search_kernel<D><<<static_cast<unsigned>(N) * H, kDecThreads, kSearchSmem, stream>>>(
+      mks, static_cast<const __nv_bfloat16*>(q), lens, Lmax, H, Hkv, BN, S, sl2, tau, w.scores, Lmax / S, count, idx,
+      w.bits, Nbm, W, g.status, g.limit_ns);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   using C = DecAttnCfg<BN, D>;
   static std::atomic<uint64_t> smem_set{0};
   if ((e = set_smem_limit_once(decode_attn_kernel<BN, D>, C::kSmem, smem_set)) != cudaSuccess) return e;
