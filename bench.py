@@ -514,29 +514,50 @@ def measure_decode(args, rr, cfg, tau, qd, kd, vd, dev, stream):
         torch.cuda.synchronize(dev)
         return e0.elapsed_time(e1) / reps
 
+    cnt_g, idx_g = torch.empty_like(cnt), torch.empty_like(idx)
+
+    def timed_g(c_, i_, reps=10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            rr.decode(qq, kc, vc, ld, B, S, tau, out=out, count=c_, idx=i_, ws=ws, stream=stream,
+                      flags=rr.VAR_GQA_MASK)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
     for _ in range(3):
         timed(tau, cnt, idx, 1)
         timed(1.0, cnt1, idx1, 1)
-    sp, de = [], []
+        timed_g(cnt_g, idx_g, 1)
+    sp, de, gp = [], [], []
     for _ in range(3):
         sp.append(timed(tau, cnt, idx))
         de.append(timed(1.0, cnt1, idx1))
+        gp.append(timed_g(cnt_g, idx_g))
     if rr.check_status(ws) != rr.RR_OK:
         raise RuntimeError("device-side status of the decode step")
-    ms, dense_ms = statistics.median(sp), statistics.median(de)
-    c_h, i_h = cnt.cpu().numpy(), idx.cpu().numpy()
-    byts = decode_bytes(cfg, lens, c_h, i_h)
-    gbs = byts["total"] / (ms / 1e3) / 1e9
+    ms, dense_ms, g_ms = statistics.median(sp), statistics.median(de), statistics.median(gp)
     peak = measured_peaks()["hbm_gbs"]
-    visited = float(c_h.sum()) / sum(H * ((ln - 1) // B + 1) for ln in lens)
+    causal = sum(H * ((ln - 1) // B + 1) for ln in lens)
+
+    def summary(c_t, i_t, t_ms):
+        c_h, i_h = c_t.cpu().numpy(), i_t.cpu().numpy()
+        byts = decode_bytes(cfg, lens, c_h, i_h)
+        gbs = byts["total"] / (t_ms / 1e3) / 1e9
+        return {"us_per_step": t_ms * 1e3, "speedup_vs_dense": dense_ms / t_ms,
+                "visited_fraction": float(c_h.sum()) / causal,
+                "hbm": {"bytes": byts["total"], "gbs": gbs, "frac_of_hbm": gbs / peak, "peak_gbs": peak,
+                        "parts": byts}}
+
+    res = {"what": "rr_decode: one new token per sequence over its KV cache (search, block-sparse attention, "
+                   "combine); caches are copies of this layer, sequence n holds L - 1000 n keys",
+           "batch": Nd, "dense_us_per_step": dense_ms * 1e3}
+    res.update(summary(cnt, idx, ms))
+    res["gqa_mask"] = summary(cnt_g, idx_g, g_ms)
     del kc, vc, ws
     torch.cuda.empty_cache()
-    return {"what": "rr_decode: one new token per sequence over its KV cache (search, block-sparse attention, "
-                    "combine); caches are copies of this layer, sequence n holds L - 1000 n keys",
-            "batch": Nd, "us_per_step": ms * 1e3, "dense_us_per_step": dense_ms * 1e3,
-            "speedup_vs_dense": dense_ms / ms, "visited_fraction": visited,
-            "hbm": {"bytes": byts["total"], "gbs": gbs, "frac_of_hbm": gbs / peak, "peak_gbs": peak,
-                    "parts": byts}}
+    return res
 
 
 def run_decode_only(args, cfg, tau):

@@ -24,7 +24,8 @@ RR_OK, RR_EINVAL, RR_EUNSUPPORTED, RR_EALIGN, RR_ECUDA, RR_ETIMEOUT, RR_ESCRATCH
 EXPORTS = ("rr_workspace_size", "rr_search", "rr_sparse_attn", "rr_attention", "rr_check_status",
            "rr_set_wait_limit_ns", "rr_status_string", "rr_search_static", "rr_mask_recall",
            "rr_workspace_size_variant", "rr_search_variant", "rr_mask_to_dense",
-           "rr_workspace_size_host", "rr_attention_host", "rr_decode_workspace_size", "rr_decode")
+           "rr_workspace_size_host", "rr_attention_host", "rr_decode_workspace_size", "rr_decode",
+           "rr_decode_variant")
 
 # sampling-variant flags of rr_search_variant (rr.h)
 VAR_ROTATE, VAR_MEAN_KEYS, VAR_GQA_MASK = 1, 2, 4
@@ -71,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.rr_decode_workspace_size.restype = ctypes.c_int
         L.rr_decode.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, vp, sz, vp]
         L.rr_decode.restype = ctypes.c_int
+        L.rr_decode_variant.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, ctypes.c_uint, vp, vp, vp, vp, sz, vp]
+        L.rr_decode_variant.restype = ctypes.c_int
         L.rr_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.rr_set_wait_limit_ns.restype = ctypes.c_uint64
         L.rr_status_string.argtypes = [i]
@@ -287,9 +290,10 @@ def decode_workspace_size(N: int, Lmax: int, H: int, Hkv: int, d: int, B: int, S
 
 
 def decode(q, k_cache, v_cache, lens, B: int, S: int, tau: float, out=None, count=None, idx=None, ws=None,
-           stream=None):
+           stream=None, flags: int = 0):
     """One decode step: q [N, H, d], caches [N, Lmax, Hkv, d] bf16, lens [N] int32
-    (device) -> (o [N, H, d], count [N, H], idx [N, H, Lmax/B])."""
+    (device) -> (o [N, H, d], count [N, H], idx [N, H, Lmax/B]).  flags:
+    VAR_GQA_MASK for one list per GQA group (rr_decode_variant)."""
     if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
         raise ValueError("q must be [N, H, d], k_cache and v_cache [N, Lmax, Hkv, d]")
     N, H, d = q.shape
@@ -308,8 +312,8 @@ def decode(q, k_cache, v_cache, lens, B: int, S: int, tau: float, out=None, coun
         idx = torch.empty((N, H, Nb), dtype=torch.int32, device=dev)
     if ws is None:
         ws = torch.empty(decode_workspace_size(N, Lmax, H, Hkv, d, B, S), dtype=torch.uint8, device=dev)
-    _check(lib().rr_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), lens.data_ptr(), N, Lmax, H, Hkv,
-                           d, B, S, float(tau), count.data_ptr(), idx.data_ptr(), out.data_ptr(), ws.data_ptr(),
-                           ws.numel(), _stream(stream)), "rr_decode")
+    _check(lib().rr_decode_variant(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), lens.data_ptr(), N, Lmax,
+                                   H, Hkv, d, B, S, float(tau), int(flags), count.data_ptr(), idx.data_ptr(),
+                                   out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)), "rr_decode_variant")
     return out, count, idx
 

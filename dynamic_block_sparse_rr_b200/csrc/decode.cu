@@ -115,12 +115,105 @@ struct DecSearchShared {
   uint32_t bits[kMaxBlocks / 32];
 };
 
+// Top-tau over the nb = Jt + 1 block masses in sh.mass, as in prefill (fixed-point
+// units of the row total, the threshold by bisection over the mass bits with
+// block-wide sums, equal masses to the lower J), plus the current block Jt.
+// The ascending list goes to rep consecutive rows of out (row stride
+// out_stride), the bitmap to rep consecutive rows of obits (W words each), the
+// count to count[0 .. rep).  Called by every thread of the CTA.
+__device__ __noinline__ void block_select(DecSearchShared& sh, int nb, int Jt, float tau, int32_t* out,
+                                          long long out_stride, uint32_t* obits, int W, int32_t* count, int rep) {
+  const int tid = threadIdx.x;
+  for (int w = tid; w < (nb + 31) / 32; w += kDecThreads) sh.bits[w] = 0u;
+  __syncthreads();
+  // this thread's contiguous chunk of the row
+  const int per = (nb + kDecThreads - 1) / kDecThreads;
+  const int c0 = min(tid * per, nb), c1 = min(c0 + per, nb);
+  uint32_t key[kMaxPer];
+  double local = 0.0;
+#pragma unroll
+  for (int e = 0; e < kMaxPer; ++e) {
+    key[e] = 0u;
+    if (c0 + e < c1) {
+      const float v = sh.mass[c0 + e];
+      key[e] = __float_as_uint(v);
+      local += static_cast<double>(v);
+    }
+  }
+  uint32_t sel_bits = 0;
+  if (tau < 1.0f) {
+    const double total = block_sum<double>(local, sh.dbuf);
+    const double scale = total > 0.0 ? 2147483648.0 / total : 0.0;
+    auto units = [&](uint32_t kk) { return __double2uint_rn(static_cast<double>(__uint_as_float(kk)) * scale); };
+    uint32_t un[kMaxPer], lsum = 0;
+#pragma unroll
+    for (int e = 0; e < kMaxPer; ++e) {
+      un[e] = c0 + e < c1 ? units(key[e]) : 0u;
+      lsum += un[e];
+    }
+    const uint32_t total_i = block_sum<uint32_t>(lsum, sh.ubuf);
+    if (total_i != 0) {
+      const uint32_t target = static_cast<uint32_t>(
+          fmin(ceil(static_cast<double>(tau) * static_cast<double>(total_i)), static_cast<double>(total_i)));
+      // the largest mass T whose masses at or above it still reach the target
+      uint32_t P = 0;
+      for (int b = 30; b >= 0; --b) {
+        const uint32_t cand = P | (1u << b);
+        uint32_t sge = 0;
+#pragma unroll
+        for (int e = 0; e < kMaxPer; ++e) sge += key[e] >= cand ? un[e] : 0u;
+        if (block_sum<uint32_t>(sge, sh.ubuf) >= target) P = cand;
+      }
+      const uint32_t T = P;
+      uint32_t sgt = 0, my_eq = 0;
+#pragma unroll
+      for (int e = 0; e < kMaxPer; ++e) {
+        sgt += key[e] > T ? un[e] : 0u;
+        my_eq += (c0 + e < c1 && key[e] == T) ? 1u : 0u;
+      }
+      const uint32_t sum_gt = block_sum<uint32_t>(sgt, sh.ubuf);
+      const uint32_t t_val = units(T);
+      const uint32_t k_eq = t_val > 0 ? (target - sum_gt + t_val - 1) / t_val : 1u;
+      uint32_t tot_eq;
+      uint32_t rank = block_excl_scan(my_eq, sh.ubuf, &tot_eq);   // masses equal to T: lowest J first
+#pragma unroll
+      for (int e = 0; e < kMaxPer; ++e) {
+        if (c0 + e < c1) {
+          bool s = key[e] > T;
+          if (key[e] == T) s = rank++ < k_eq;
+          if (s) sel_bits |= 1u << e;
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kMaxPer; ++e)
+      if (c0 + e < c1) sel_bits |= 1u << e;
+  }
+  if (Jt >= c0 && Jt < c1) sel_bits |= 1u << (Jt - c0);   // the block holding the query
+  uint32_t my_sel = __popc(sel_bits), cnt;
+  uint32_t pos = block_excl_scan(my_sel, sh.ubuf, &cnt);
+#pragma unroll
+  for (int e = 0; e < kMaxPer; ++e) {
+    if (sel_bits & (1u << e)) {
+      for (int r = 0; r < rep; ++r) out[r * out_stride + pos] = c0 + e;
+      ++pos;
+      atomicOr(&sh.bits[(c0 + e) >> 5], 1u << ((c0 + e) & 31));
+    }
+  }
+  __syncthreads();
+  for (int r = 0; r < rep; ++r)
+    for (int w = tid; w < W; w += kDecThreads) obits[r * W + w] = w < (nb + 31) / 32 ? sh.bits[w] : 0u;
+  if (tid < rep) count[tid] = static_cast<int32_t>(cnt);
+}
+
+
 template <int D>
 __global__ void __launch_bounds__(kDecThreads) decode_search_kernel(
     const __grid_constant__ CUtensorMap mks, const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lens,
     int Lmax, int H, int Hkv, int B, int S, float sl2, float tau, float* __restrict__ scores, int Ns_max,
     int32_t* __restrict__ count, int32_t* __restrict__ idx, uint32_t* __restrict__ bits, int Nbm, int W,
-    unsigned int* status, uint64_t limit_ns) {
+    float* __restrict__ group_mass, unsigned int* status, uint64_t limit_ns) {
   constexpr int kTileBytes = kSearchTile * D * 2;
   __shared__ DecSearchShared sh;
   extern __shared__ uint8_t smem_raw[];
@@ -224,86 +317,48 @@ __global__ void __launch_bounds__(kDecThreads) decode_search_kernel(
     for (int j = J * r; j < j1; ++j) m += exp2f(sc[j] - mx);
     sh.mass[J] = m;
   }
-  for (int w = tid; w < (nb + 31) / 32; w += kDecThreads) sh.bits[w] = 0u;
   __syncthreads();
 
-  // Top-tau over J <= Jt: this thread's contiguous chunk of the row
-  const int per = (nb + kDecThreads - 1) / kDecThreads;
-  const int c0 = min(tid * per, nb), c1 = min(c0 + per, nb);
-  uint32_t key[kMaxPer];
-  double local = 0.0;
-#pragma unroll
-  for (int e = 0; e < kMaxPer; ++e) {
-    key[e] = 0u;
-    if (c0 + e < c1) {
-      const float v = sh.mass[c0 + e];
-      key[e] = __float_as_uint(v);
-      local += static_cast<double>(v);
-    }
+  if (group_mass) {   // one mask per GQA group: the head's masses, normalised, for the group kernel
+    float lsum = 0.f;
+    for (int J = tid; J < nb; J += kDecThreads) lsum += sh.mass[J];
+    const float tot = block_sum<float>(lsum, sh.fbuf);
+    const float inv = tot > 0.f ? 1.0f / tot : 0.f;
+    float* mrow = group_mass + row * Nbm;
+    for (int J = tid; J < nb; J += kDecThreads) mrow[J] = sh.mass[J] * inv;
+    return;
   }
-  uint32_t sel_bits = 0;
-  if (tau < 1.0f) {
-    const double total = block_sum<double>(local, sh.dbuf);
-    const double scale = total > 0.0 ? 2147483648.0 / total : 0.0;
-    auto units = [&](uint32_t kk) { return __double2uint_rn(static_cast<double>(__uint_as_float(kk)) * scale); };
-    uint32_t un[kMaxPer], lsum = 0;
-#pragma unroll
-    for (int e = 0; e < kMaxPer; ++e) {
-      un[e] = c0 + e < c1 ? units(key[e]) : 0u;
-      lsum += un[e];
-    }
-    const uint32_t total_i = block_sum<uint32_t>(lsum, sh.ubuf);
-    if (total_i != 0) {
-      const uint32_t target = static_cast<uint32_t>(
-          fmin(ceil(static_cast<double>(tau) * static_cast<double>(total_i)), static_cast<double>(total_i)));
-      // the largest mass T whose masses at or above it still reach the target
-      uint32_t P = 0;
-      for (int b = 30; b >= 0; --b) {
-        const uint32_t cand = P | (1u << b);
-        uint32_t sge = 0;
-#pragma unroll
-        for (int e = 0; e < kMaxPer; ++e) sge += key[e] >= cand ? un[e] : 0u;
-        if (block_sum<uint32_t>(sge, sh.ubuf) >= target) P = cand;
-      }
-      const uint32_t T = P;
-      uint32_t sgt = 0, my_eq = 0;
-#pragma unroll
-      for (int e = 0; e < kMaxPer; ++e) {
-        sgt += key[e] > T ? un[e] : 0u;
-        my_eq += (c0 + e < c1 && key[e] == T) ? 1u : 0u;
-      }
-      const uint32_t sum_gt = block_sum<uint32_t>(sgt, sh.ubuf);
-      const uint32_t t_val = units(T);
-      const uint32_t k_eq = t_val > 0 ? (target - sum_gt + t_val - 1) / t_val : 1u;
-      uint32_t tot_eq;
-      uint32_t rank = block_excl_scan(my_eq, sh.ubuf, &tot_eq);   // masses equal to T: lowest J first
-#pragma unroll
-      for (int e = 0; e < kMaxPer; ++e) {
-        if (c0 + e < c1) {
-          bool s = key[e] > T;
-          if (key[e] == T) s = rank++ < k_eq;
-          if (s) sel_bits |= 1u << e;
-        }
-      }
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < kMaxPer; ++e)
-      if (c0 + e < c1) sel_bits |= 1u << e;
+  block_select(sh, nb, Jt, tau, out, Nbm, obits, W, count + row, 1);
+}
+
+// One mask per GQA group (decode): the block masses of the group's g heads,
+// written by the search kernels, summed in head order; the selection goes to
+// every head of the group.  One CTA per (sequence, kv head).
+__global__ void __launch_bounds__(kDecThreads) decode_group_select_kernel(const float* __restrict__ group_mass,
+                                                                         const int32_t* __restrict__ lens, int Lmax,
+                                                                         int H, int Hkv, int B, float tau,
+                                                                         int32_t* __restrict__ count,
+                                                                         int32_t* __restrict__ idx,
+                                                                         uint32_t* __restrict__ bits, int Nbm, int W) {
+  __shared__ DecSearchShared sh;
+  const int tid = threadIdx.x;
+  const int n = static_cast<int>(blockIdx.x) / Hkv, kvh = static_cast<int>(blockIdx.x) % Hkv;
+  const int g = H / Hkv;
+  const long long row0 = static_cast<long long>(n) * H + kvh * g;   // first head of the group
+  const int len = __ldg(lens + n);
+  if (len < 1 || len > Lmax) {   // the search recorded it; nothing selected
+    if (tid < g) count[row0 + tid] = 0;
+    for (int i = tid; i < g * W; i += kDecThreads) bits[row0 * W + i] = 0u;
+    return;
   }
-  if (Jt >= c0 && Jt < c1) sel_bits |= 1u << (Jt - c0);   // the block holding the query
-  uint32_t my_sel = __popc(sel_bits), cnt;
-  uint32_t pos = block_excl_scan(my_sel, sh.ubuf, &cnt);
-#pragma unroll
-  for (int e = 0; e < kMaxPer; ++e) {
-    if (sel_bits & (1u << e)) {
-      out[pos++] = c0 + e;
-      atomicOr(&sh.bits[(c0 + e) >> 5], 1u << ((c0 + e) & 31));
-    }
+  const int Jt = (len - 1) / B, nb = Jt + 1;
+  for (int J = tid; J < nb; J += kDecThreads) {
+    float m = 0.f;
+    for (int r = 0; r < g; ++r) m += group_mass[(row0 + r) * Nbm + J];
+    sh.mass[J] = m;
   }
   __syncthreads();
-  for (int w = tid; w < W; w += kDecThreads) obits[w] = w < (nb + 31) / 32 ? sh.bits[w] : 0u;
-  if (tid == 0) count[row] = static_cast<int32_t>(cnt);
+  block_select(sh, nb, Jt, tau, idx + row0 * Nbm, Nbm, bits + row0 * W, W, count + row0, g);
 }
 
 // ------------------------------------------------------------------ attention
@@ -605,7 +660,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restri
 
 template <int BN, int D>
 cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const int32_t* lens, int N, int Lmax, int H,
-                            int Hkv, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                            int Hkv, int S, float tau, bool gqa, int32_t* count, int32_t* idx, void* o,
                             const DecodeScratch& w, const DeviceGuardArgs& g, cudaStream_t stream) {
   const int Nbm = Lmax / BN, W = (Nbm + 31) / 32;
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
@@ -620,8 +675,13 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
   if (e != cudaSuccess) return e;
   decode_search_kernel<D><<<static_cast<unsigned>(N) * H, kDecThreads, kSearchSmem, stream>>>(
       mks, static_cast<const __nv_bfloat16*>(q), lens, Lmax, H, Hkv, BN, S, sl2, tau, w.scores, Lmax / S, count, idx,
-      w.bits, Nbm, W, g.status, g.limit_ns);
+      w.bits, Nbm, W, gqa ? w.mass : nullptr, g.status, g.limit_ns);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (gqa) {
+    decode_group_select_kernel<<<static_cast<unsigned>(N) * Hkv, kDecThreads, 0, stream>>>(
+        w.mass, lens, Lmax, H, Hkv, BN, tau, count, idx, w.bits, Nbm, W);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   using C = DecAttnCfg<BN, D>;
   static std::atomic<uint64_t> smem_set{0};
   if ((e = set_smem_limit_once(decode_attn_kernel<BN, D>, C::kSmem, smem_set)) != cudaSuccess) return e;
@@ -637,12 +697,12 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
 }  // namespace
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const int32_t* lens, int N, int Lmax, int H,
-                          int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                          int Hkv, int d, int B, int S, float tau, bool gqa, int32_t* count, int32_t* idx, void* o,
                           const DecodeScratch& w, const DeviceGuardArgs& g, cudaStream_t stream) {
-  if (B == 128 && d == 128) return launch_decode_t<128, 128>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, count, idx, o, w, g, stream);
-  if (B == 128 && d == 64) return launch_decode_t<128, 64>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, count, idx, o, w, g, stream);
-  if (B == 64 && d == 128) return launch_decode_t<64, 128>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, count, idx, o, w, g, stream);
-  if (B == 64 && d == 64) return launch_decode_t<64, 64>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, count, idx, o, w, g, stream);
+  if (B == 128 && d == 128) return launch_decode_t<128, 128>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, gqa, count, idx, o, w, g, stream);
+  if (B == 128 && d == 64) return launch_decode_t<128, 64>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, gqa, count, idx, o, w, g, stream);
+  if (B == 64 && d == 128) return launch_decode_t<64, 128>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, gqa, count, idx, o, w, g, stream);
+  if (B == 64 && d == 64) return launch_decode_t<64, 64>(q, k, v, lens, N, Lmax, H, Hkv, S, tau, gqa, count, idx, o, w, g, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -136,7 +136,7 @@ HostLayout carve_host(int L, int H, int Hkv, int d, int B, int S) {
 // kept-block bitmaps [N, H, W] u32 (W = ceil(Lmax/B / 32)) and the attention
 // partials [N, H, NC, d+2] fp32, one per 16-block chunk (NC = ceil(Lmax/B / 16)).
 struct DecodeLayout {
-  size_t status, scores, bits, part, total;
+  size_t status, scores, bits, part, mass, total;
 };
 
 DecodeLayout carve_decode(int N, int Lmax, int H, int d, int B, int S) {
@@ -149,6 +149,7 @@ DecodeLayout carve_decode(int N, int Lmax, int H, int d, int B, int S) {
   w.scores = off; off += round_up(rows * (Lmax / S) * 4);
   w.bits = off; off += round_up(rows * W * 4);
   w.part = off; off += round_up(rows * NC * (d + 2) * 4);
+  w.mass = off; off += round_up(rows * static_cast<size_t>(Lmax / B) * 4);
   w.total = off;
   return w;
 }
@@ -377,9 +378,10 @@ rr_status rr_decode_workspace_size(int N, int Lmax, int H, int Hkv, int d, int B
   return RR_OK;
 }
 
-rr_status rr_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int N, int Lmax,
-                    int H, int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
-                    void* workspace, size_t workspace_bytes, void* stream) {
+rr_status rr_decode_variant(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int N,
+                            int Lmax, int H, int Hkv, int d, int B, int S, float tau, unsigned flags, int32_t* count,
+                            int32_t* idx, void* o, void* workspace, size_t workspace_bytes, void* stream) {
+  if (flags & ~static_cast<unsigned>(RR_VAR_GQA_MASK)) return RR_EINVAL;
   rr_status st = check_decode_shape(N, Lmax, H, Hkv, d, B, S);
   if (st != RR_OK) return st;
   if (!(tau > 0.0f) || tau != tau) return RR_EINVAL;
@@ -395,13 +397,20 @@ rr_status rr_decode(const void* q, const void* k_cache, const void* v_cache, con
   unsigned int* status = reinterpret_cast<unsigned int*>(ws + w.status);
   const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
   const rr::DecodeScratch sc{reinterpret_cast<float*>(ws + w.scores), reinterpret_cast<uint32_t*>(ws + w.bits),
-                             reinterpret_cast<float*>(ws + w.part)};
+                             reinterpret_cast<float*>(ws + w.part), reinterpret_cast<float*>(ws + w.mass)};
   const Range range("rr_decode");
   if (cudaMemsetAsync(status, 0, sizeof(unsigned int), s) != cudaSuccess) return RR_ECUDA;
-  if (rr::launch_decode(q, k_cache, v_cache, lens, N, Lmax, H, Hkv, d, B, S, tau, count, idx, o, sc, g, s) !=
-      cudaSuccess)
+  if (rr::launch_decode(q, k_cache, v_cache, lens, N, Lmax, H, Hkv, d, B, S, tau, (flags & RR_VAR_GQA_MASK) != 0,
+                        count, idx, o, sc, g, s) != cudaSuccess)
     return RR_ECUDA;
   return RR_OK;
+}
+
+rr_status rr_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int N, int Lmax,
+                    int H, int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  return rr_decode_variant(q, k_cache, v_cache, lens, N, Lmax, H, Hkv, d, B, S, tau, 0u, count, idx, o, workspace,
+                           workspace_bytes, stream);
 }
 
 rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int Nb, uint8_t* dense, void* stream) {

@@ -98,12 +98,14 @@ struct DecodeScratch {
   float* scores;
   uint32_t* bits;
   float* part;
+  float* mass;   // per-head block masses [N, H, Lmax/B] fp32 (one mask per GQA group only)
 };
 
 // Decode stage: search, block-sparse attention and combine for one new token per
 // sequence.  q, o: [N, H, d]; k, v: [N, Lmax, Hkv, d]; lens: [N] cache lengths.
+// gqa: one mask per GQA group, selected on the group's summed block mass.
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const int32_t* lens, int N, int Lmax, int H,
-                          int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
+                          int Hkv, int d, int B, int S, float tau, bool gqa, int32_t* count, int32_t* idx, void* o,
                           const DecodeScratch& w, const DeviceGuardArgs& g, cudaStream_t stream);
 
 // Largest Nb = L/B the kernels accept (bounded by the on-chip list / sort buffers).

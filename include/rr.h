@@ -203,7 +203,8 @@ rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int 
  * Out: count [N,H] int32, idx [N,H,Lmax/B] int32 (kept blocks ascending, valid
  *      below count), o [N,H,d] bf16.  All device memory, caller-owned.
  * Workspace: rr_decode_workspace_size bytes, 256-byte aligned (sampled scores,
- * kept-block bitmaps, per-chunk attention partials, status word).
+ * kept-block bitmaps, per-chunk attention partials, per-head block masses,
+ * status word).
  * Requires Lmax % B == 0, B % S == 0, d and B in {64, 128}, H/Hkv <= 8,
  * Lmax/B <= 4096.  A length outside [1, Lmax] is found on the device: that
  * sequence gets count 0 and a zero output, and rr_check_status returns
@@ -215,6 +216,18 @@ rr_status rr_decode_workspace_size(int N, int Lmax, int H, int Hkv, int d, int B
 rr_status rr_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int N, int Lmax,
                     int H, int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* The decode step with the search's sampling variants: flags 0 is rr_decode;
+ * RR_VAR_GQA_MASK keeps one list per GQA group, selected (Top-tau plus the
+ * current block) on the sum of the group's per-head block masses (each head's
+ * normalised to 1), and every head of the group receives it.  A kept block is
+ * loaded once for its whole group either way, so with per-head lists the bytes
+ * read follow the union of the group's lists, with this flag the group's own
+ * selection.  Other flag bits: RR_EINVAL.  Workspace, arguments and outputs as
+ * rr_decode. */
+rr_status rr_decode_variant(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int N,
+                            int Lmax, int H, int Hkv, int d, int B, int S, float tau, unsigned flags, int32_t* count,
+                            int32_t* idx, void* o, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, returns the device-side status recorded since the
  * last rr_* call that started on this workspace (RR_OK, RR_ETIMEOUT, RR_EMASK,

@@ -375,10 +375,22 @@ def decode_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, t: int, blocks
     return out
 
 
-def rr_decode(q: np.ndarray, K: np.ndarray, V: np.ndarray, t: int, B: int, S: int, tau: float):
+def decode_group_mass(M: np.ndarray, Hkv: int) -> np.ndarray:
+    """V3 for the decode step: the block masses of the g query heads of each kv
+    head summed, repeated for every head of the group.  [H, J_t + 1]."""
+    H, n = M.shape
+    g = H // Hkv
+    return np.repeat(M.reshape(Hkv, g, n).sum(axis=1), g, axis=0)
+
+
+def rr_decode(q: np.ndarray, K: np.ndarray, V: np.ndarray, t: int, B: int, S: int, tau: float,
+              gqa_mask: bool = False):
     """One decode step of one sequence (D1-D5): returns (count [H], idx list per
-    head, normalised mass [H, J_t + 1], output [H, d])."""
+    head, the mass the selection ran on [H, J_t + 1], output [H, d]).  gqa_mask
+    (V3): one list per GQA group, selected on the group's summed mass."""
     M = decode_block_mass(q, K, t, B, S)
+    if gqa_mask:
+        M = decode_group_mass(M, K.shape[1])
     Jt = t // B
     sel = [decode_select(M[h], Jt, tau) for h in range(q.shape[0])]
     count = np.array([x.size for x in sel], dtype=np.int32)

@@ -212,4 +212,9 @@ def test_decode_workspace_and_rejections(rr):
     assert call(lens=g + 2) == rr.RR_EALIGN
     assert call(ws=g + 16) == rr.RR_EALIGN
     assert call(nws=nws - 1) == rr.RR_EINVAL
+    # the decode variants take only the GQA-mask flag
+    assert lib.rr_decode_variant(g, g, g, g, N, Lmax, H, Hkv, d, B, S, 0.9, rr.VAR_ROTATE, g, g, g, g, nws,
+                                 None) == rr.RR_EINVAL
+    assert lib.rr_decode_variant(g, g, g, g, N, Lmax, H, Hkv, d, B, S, 0.0, rr.VAR_GQA_MASK, g, g, g, g, nws,
+                                 None) == rr.RR_EINVAL
 

@@ -44,13 +44,14 @@ def _make(N, Lmax, H, Hkv, d, structure, seed):
     return qs, np.stack(ks), np.stack(vs)
 
 
-def run_case(rr, N, Lmax, H, Hkv, d, B, S, tau, lens, structure=gen.PLANTED, seed=0):
+def run_case(rr, N, Lmax, H, Hkv, d, B, S, tau, lens, structure=gen.PLANTED, seed=0, flags=0):
     Qs, K, V = _make(N, Lmax, H, Hkv, d, structure, seed)
     q = np.stack([Qs[n][lens[n] - 1] for n in range(N)])              # [N, H, d]
     qd, kd, vd = _bf16(q).cuda(), _bf16(K).cuda(), _bf16(V).cuda()
     ld = torch.tensor(lens, dtype=torch.int32, device="cuda")
     ws = torch.empty(rr.decode_workspace_size(N, Lmax, H, Hkv, d, B, S), dtype=torch.uint8, device="cuda")
-    o, count, idx = rr.decode(qd, kd, vd, ld, B, S, tau, ws=ws)
+    o, count, idx = rr.decode(qd, kd, vd, ld, B, S, tau, ws=ws, flags=flags)
+    gqa = bool(flags & rr.VAR_GQA_MASK)
     assert rr.check_status(ws) == rr.RR_OK
     count, idx, og = count.cpu().numpy(), idx.cpu().numpy(), o.float().cpu().numpy()
     stats = {"rows_differing": 0, "band": 0, "tie": 0, "fail": 0}
@@ -59,6 +60,12 @@ def run_case(rr, N, Lmax, H, Hkv, d, B, S, tau, lens, structure=gen.PLANTED, see
         t = lens[n] - 1
         Jt = t // B
         M = oracle.decode_block_mass(q[n], K[n], t, B, S)
+        if gqa:
+            M = oracle.decode_group_mass(M, Hkv)
+            g = H // Hkv
+            for h in range(H):
+                c0 = (h // g) * g
+                assert count[n, h] == count[n, c0] and np.array_equal(idx[n, h, :count[n, h]], idx[n, c0, :count[n, c0]])
         blocks = []
         for h in range(H):
             g_sel = idx[n, h, :count[n, h]]
@@ -105,6 +112,17 @@ def test_decode_block_and_head_sizes(rr, B, d, S):
 def test_decode_gqa_seven_to_one_video(rr):
     lens = [4096, 2500]
     run_case(rr, 2, 4096, 7, 1, 128, 128, 16, 0.95, lens, structure=gen.VIDEO, seed=5)
+
+
+@pytest.mark.parametrize("structure,H,Hkv,tau", [(gen.PLANTED, 8, 2, 0.9), (gen.VIDEO, 7, 1, 0.95),
+                                                  (gen.PLANTED_BAND, 4, 4, 0.8)])
+def test_decode_gqa_group_mask(rr, structure, H, Hkv, tau):
+    """One list per GQA group (rr_decode_variant, RR_VAR_GQA_MASK): selected on the
+    group's summed mass, the same on every head of the group; with one head per
+    group it is the per-head list."""
+    lens = [4096, 3001, 200, 1]
+    run_case(rr, len(lens), 4096, H, Hkv, 128, 128, 16, tau, lens, structure=structure, seed=17,
+             flags=rr.VAR_GQA_MASK)
 
 
 def test_decode_tau_one_is_dense(rr):

@@ -154,6 +154,32 @@ def test_decode_row_matches_prefill_row_when_the_query_is_sampled():
             assert np.allclose(Md[h], Mp[h, i, :i + 1], atol=1e-12), (h, i)
 
 
+def test_group_mask_shares_lists_and_reaches_tau():
+    """V3 for decode: every head of a GQA group gets the list selected on the
+    group's summed mass; it reaches tau of that mass, keeps the current block,
+    and with one head per group it is the per-head list."""
+    L, H, Hkv, d, B, S, tau = 512, 8, 2, 16, 32, 4, 0.8
+    rng = np.random.default_rng(12)
+    q, K, V = 2.0 * rng.standard_normal((H, d)), rng.standard_normal((L, Hkv, d)), rng.standard_normal((L, Hkv, d))
+    t = 450
+    Jt = t // B
+    count, sel, Mg, _ = oracle.rr_decode(q, K, V, t, B, S, tau, gqa_mask=True)
+    M = oracle.decode_block_mass(q, K, t, B, S)
+    g = H // Hkv
+    for c in range(Hkv):
+        grp = M[c * g:(c + 1) * g].sum(axis=0)
+        for h in range(c * g, (c + 1) * g):
+            assert np.array_equal(sel[h], sel[c * g])
+            assert np.allclose(Mg[h], grp, atol=1e-14)
+        m = grp / grp.sum()
+        assert Jt in sel[c * g] and m[sel[c * g]].sum() >= tau
+    # one head per group: the group mask is the per-head mask
+    K8 = np.repeat(K, 4, axis=1)
+    c1, s1, _, o1 = oracle.rr_decode(q, K8, np.repeat(V, 4, axis=1), t, B, S, tau, gqa_mask=True)
+    c2, s2, _, o2 = oracle.rr_decode(q, K8, np.repeat(V, 4, axis=1), t, B, S, tau)
+    assert all(np.array_equal(a, b) for a, b in zip(s1, s2)) and np.allclose(o1, o2)
+
+
 # ------------------------------------------------------------ planted mistakes
 _orig = {n: getattr(oracle, n) for n in ("decode_positions", "decode_select", "decode_attention")}
 
