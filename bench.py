@@ -550,8 +550,8 @@ def measure_decode(args, rr, cfg, tau, qd, kd, vd, dev, stream):
                 "hbm": {"bytes": byts["total"], "gbs": gbs, "frac_of_hbm": gbs / peak, "peak_gbs": peak,
                         "parts": byts}}
 
-    res = {"what": "rr_decode: one new token per sequence over its KV cache (search, block-sparse attention, "
-                   "combine); caches are copies of this layer, sequence n holds L - 1000 n keys",
+    res = {"what": "rr_decode: one new token per sequence over its KV cache (search, block-sparse attention "
+                   "with the partials merged); caches are copies of this layer, sequence n holds L - 1000 n keys",
            "batch": Nd, "dense_us_per_step": dense_ms * 1e3}
     res.update(summary(cnt, idx, ms))
     res["gqa_mask"] = summary(cnt_g, idx_g, g_ms)

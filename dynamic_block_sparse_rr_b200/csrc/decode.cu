@@ -11,27 +11,36 @@
 //
 // The path is bound by HBM (the sampled keys, then the kept K and V blocks); the
 // kernels are sized for bytes in flight and kept lean in instructions:
-//   decode_search_kernel   one CTA per (sequence, head): the head's sampled key
-//                          rows come in as 128-row TMA tiles of a zero-copy
-//                          strided view (two-stage ring), scores to the
-//                          workspace, block mass in shared memory, Top-tau by
-//                          bisection over the
-//                          mass bits with block-wide sums of fixed-point units
-//                          (the prefill rule), list and a bitmap of the kept
-//                          blocks out;
-//   decode_attn_kernel     one CTA per (sequence, kv head, 16 key blocks): a
-//                          kept block's K and V tiles come in once by TMA
-//                          (three-stage ring) for every query head of the GQA
-//                          group that kept it.  The group's <= 8 heads are the 8
-//                          columns of m16n8k16 tensor-core tiles (mma.sync), so
-//                          the two small contractions per block (scores of 128
-//                          keys, P V) are a few instructions per warp; each warp
-//                          keeps an online softmax over its 16 keys of every
-//                          block, and the warps' partials merge into the
-//                          chunk's partial (max, sum, output);
-//   decode_combine_kernel  one CTA per (sequence, head): the partials merged.
+//   decode_search_kernel   a few CTAs per (sequence, head), each over a run of
+//                          the head's sampled key rows: 128-row TMA tiles of a
+//                          zero-copy strided view (two-stage ring) scored on
+//                          m16n8k16 tensor-core tiles (mma.sync, q as column 0),
+//                          scores to the workspace, the run's max and block
+//                          masses on that max.  The CTA that finishes a row
+//                          last puts the row's masses on one scale and runs
+//                          Top-tau by bisection over the mass bits with
+//                          block-wide sums of fixed-point units (the prefill
+//                          rule); list and a bitmap of the kept blocks out.
+//                          One CTA also writes the prefix of the sequences'
+//                          block counts;
+//   decode_attn_kernel     one persistent CTA per SM over an equal share of the
+//                          flattened (sequence, kv head, causal key block)
+//                          space: a kept block's K and V tiles come in once by
+//                          TMA (three-stage ring, running on across rows) for
+//                          every query head of the GQA group that kept it.  The
+//                          group's <= 8 heads are the 8 columns of m16n8k16
+//                          tiles, so the two small contractions per block
+//                          (scores of 128 keys, P V) are a few instructions per
+//                          warp; each warp keeps an online softmax over its 16
+//                          keys of every block.  At the end of each row the
+//                          warps' partials merge into the CTA's partial for the
+//                          row, and the last of the row's CTAs to finish merges
+//                          those into the output.
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <algorithm>
+#include <atomic>
 
 #include "rr_internal.h"
 #include "sm100.cuh"
@@ -99,32 +108,54 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* buf, u
 constexpr int kSearchTile = 128;   // sampled keys per TMA tile of the search
 constexpr int kSearchStages = 2;
 
-// Byte offset of element (row, c) of a 128-row TMA tile (128-byte swizzle, D/64
-// column blocks of 128 rows x 128 bytes); c a multiple of 8.
-__device__ __forceinline__ uint32_t swz128(int row, int c) {
-  return static_cast<uint32_t>((c >> 6) * (128 * 128) + row * 128 + ((((c & 63) >> 3) ^ (row & 7)) << 4));
+// Byte offset of element (row, c) in a TMA tile of rows x D bf16 stored as D/64
+// column blocks of rows x 128 bytes with the 128-byte swizzle (c a multiple of 8
+// when used as a 16-byte row address).
+template <int BN>
+__device__ __forceinline__ uint32_t swz(int row, int c) {
+  return static_cast<uint32_t>((c >> 6) * (BN * 128) + row * 128 + ((((c & 63) >> 3) ^ (row & 7)) << 4) + (c & 7) * 2);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col).
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 struct DecSearchShared {
   uint64_t full[kSearchStages];
   int abort;
-  float mass[kMaxBlocks];
+  int last;
   double dbuf[kDecWarps];
   float fbuf[kDecWarps];
   uint32_t ubuf[kDecWarps];
-  uint32_t bits[kMaxBlocks / 32];
+  uint32_t hist[kDecThreads];   // radix digits of the threshold search
+  uint32_t digit, above;
 };
 
-// Top-tau over the nb = Jt + 1 block masses in sh.mass, as in prefill (fixed-point
-// units of the row total, the threshold by bisection over the mass bits with
-// block-wide sums, equal masses to the lower J), plus the current block Jt.
-// The ascending list goes to rep consecutive rows of out (row stride
+// Top-tau over the nb = Jt + 1 block masses in mass[] (shared memory), as in
+// prefill (fixed-point units of the row total, the threshold by bisection over
+// the mass bits with block-wide sums, equal masses to the lower J), plus the
+// current block Jt.  wbits (shared memory, ceil(nb/32) words) collects the
+// bitmap.  The ascending list goes to rep consecutive rows of out (row stride
 // out_stride), the bitmap to rep consecutive rows of obits (W words each), the
 // count to count[0 .. rep).  Called by every thread of the CTA.
-__device__ __noinline__ void block_select(DecSearchShared& sh, int nb, int Jt, float tau, int32_t* out,
-                                          long long out_stride, uint32_t* obits, int W, int32_t* count, int rep) {
+__device__ __noinline__ void block_select(DecSearchShared& sh, const float* mass, uint32_t* wbits, int nb, int Jt,
+                                          float tau, int32_t* out, long long out_stride, uint32_t* obits, int W,
+                                          int32_t* count, int rep) {
   const int tid = threadIdx.x;
-  for (int w = tid; w < (nb + 31) / 32; w += kDecThreads) sh.bits[w] = 0u;
+  for (int w = tid; w < (nb + 31) / 32; w += kDecThreads) wbits[w] = 0u;
   __syncthreads();
   // this thread's contiguous chunk of the row
   const int per = (nb + kDecThreads - 1) / kDecThreads;
@@ -135,7 +166,7 @@ __device__ __noinline__ void block_select(DecSearchShared& sh, int nb, int Jt, f
   for (int e = 0; e < kMaxPer; ++e) {
     key[e] = 0u;
     if (c0 + e < c1) {
-      const float v = sh.mass[c0 + e];
+      const float v = mass[c0 + e];
       key[e] = __float_as_uint(v);
       local += static_cast<double>(v);
     }
@@ -155,23 +186,34 @@ __device__ __noinline__ void block_select(DecSearchShared& sh, int nb, int Jt, f
     if (total_i != 0) {
       const uint32_t target = static_cast<uint32_t>(
           fmin(ceil(static_cast<double>(tau) * static_cast<double>(total_i)), static_cast<double>(total_i)));
-      // the largest mass T whose masses at or above it still reach the target
-      uint32_t P = 0;
-      for (int b = 30; b >= 0; --b) {
-        const uint32_t cand = P | (1u << b);
-        uint32_t sge = 0;
+      // the largest mass T whose masses at or above it still reach the target,
+      // one 8-bit digit of its bits at a time from the top: `above` holds the
+      // units of the masses above the digits fixed so far, and the digit taken
+      // is the largest whose masses, with `above`, reach the target
+      uint32_t T = 0, above = 0;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        sh.hist[tid] = 0u;
+        __syncthreads();
+        const uint32_t hmask = shift == 24 ? 0u : (0xffffffffu << (shift + 8));
 #pragma unroll
-        for (int e = 0; e < kMaxPer; ++e) sge += key[e] >= cand ? un[e] : 0u;
-        if (block_sum<uint32_t>(sge, sh.ubuf) >= target) P = cand;
+        for (int e = 0; e < kMaxPer; ++e)
+          if (c0 + e < c1 && (key[e] & hmask) == T) atomicAdd(&sh.hist[(key[e] >> shift) & 255u], un[e]);
+        __syncthreads();
+        const uint32_t v = sh.hist[255 - tid];   // thread i takes digit 255 - i
+        uint32_t all;
+        const uint32_t ex = block_excl_scan(v, sh.ubuf, &all);   // units of the digits above it
+        if (above + ex < target && above + ex + v >= target) {
+          sh.digit = 255u - tid;
+          sh.above = above + ex;
+        }
+        __syncthreads();
+        T |= sh.digit << shift;
+        above = sh.above;
       }
-      const uint32_t T = P;
-      uint32_t sgt = 0, my_eq = 0;
+      const uint32_t sum_gt = above;   // units of the masses above T
+      uint32_t my_eq = 0;
 #pragma unroll
-      for (int e = 0; e < kMaxPer; ++e) {
-        sgt += key[e] > T ? un[e] : 0u;
-        my_eq += (c0 + e < c1 && key[e] == T) ? 1u : 0u;
-      }
-      const uint32_t sum_gt = block_sum<uint32_t>(sgt, sh.ubuf);
+      for (int e = 0; e < kMaxPer; ++e) my_eq += (c0 + e < c1 && key[e] == T) ? 1u : 0u;
       const uint32_t t_val = units(T);
       const uint32_t k_eq = t_val > 0 ? (target - sum_gt + t_val - 1) / t_val : 1u;
       uint32_t tot_eq;
@@ -198,64 +240,103 @@ __device__ __noinline__ void block_select(DecSearchShared& sh, int nb, int Jt, f
     if (sel_bits & (1u << e)) {
       for (int r = 0; r < rep; ++r) out[r * out_stride + pos] = c0 + e;
       ++pos;
-      atomicOr(&sh.bits[(c0 + e) >> 5], 1u << ((c0 + e) & 31));
+      atomicOr(&wbits[(c0 + e) >> 5], 1u << ((c0 + e) & 31));
     }
   }
   __syncthreads();
   for (int r = 0; r < rep; ++r)
-    for (int w = tid; w < W; w += kDecThreads) obits[r * W + w] = w < (nb + 31) / 32 ? sh.bits[w] : 0u;
+    for (int w = tid; w < W; w += kDecThreads) obits[r * W + w] = w < (nb + 31) / 32 ? wbits[w] : 0u;
   if (tid < rep) count[tid] = static_cast<int32_t>(cnt);
 }
 
 
+// Exclusive prefix of the sequences' causal block counts (0 for a length
+// outside [1, Lmax]): rowstart[n], and rowstart[N] the total.  Called by every
+// thread of one CTA.
+__device__ void block_count_prefix(const int32_t* __restrict__ lens, int N, int Lmax, int B,
+                                   int32_t* __restrict__ rowstart, uint32_t* buf) {
+  uint32_t carry = 0;
+  for (int base = 0; base < N; base += kDecThreads) {
+    const int n = base + static_cast<int>(threadIdx.x);
+    uint32_t nbl = 0;
+    if (n < N) {
+      const int len = __ldg(lens + n);
+      nbl = (len >= 1 && len <= Lmax) ? static_cast<uint32_t>((len - 1) / B + 1) : 0u;
+    }
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan(nbl, buf, &tot);
+    if (n < N) rowstart[n] = static_cast<int32_t>(carry + ex);
+    carry += tot;
+  }
+  if (threadIdx.x == 0) rowstart[N] = static_cast<int32_t>(carry);
+}
+
+// grid (SC, N*H): CTA (c, row) scores the sampled keys of tiles [c tpc, (c+1) tpc)
+// of its (sequence, head) row and owns the key blocks those keys fall in
+// (B/S divides the 128 strides of a tile).  Its max and its blocks' masses on
+// that max go to the workspace; the CTA that arrives last on the row's counter
+// (zeroed before the launch) rescales every chunk's masses to the row max and
+// selects.
 template <int D>
-__global__ void __launch_bounds__(kDecThreads) decode_search_kernel(
+__global__ void __launch_bounds__(kDecThreads, 3) decode_search_kernel(
     const __grid_constant__ CUtensorMap mks, const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lens,
-    int Lmax, int H, int Hkv, int B, int S, float sl2, float tau, float* __restrict__ scores, int Ns_max,
+    int N, int Lmax, int H, int Hkv, int B, int S, float sl2, float tau, int tpc, float* __restrict__ scores,
+    int Ns_max, float* __restrict__ cmax, unsigned int* __restrict__ arrive, float* __restrict__ mass, int group,
     int32_t* __restrict__ count, int32_t* __restrict__ idx, uint32_t* __restrict__ bits, int Nbm, int W,
-    float* __restrict__ group_mass, unsigned int* status, uint64_t limit_ns) {
+    int32_t* __restrict__ rowstart, __nv_bfloat16* __restrict__ o, unsigned int* status, uint64_t limit_ns) {
   constexpr int kTileBytes = kSearchTile * D * 2;
+  static_assert(kMaxBlocks * 4 + kMaxBlocks / 8 <= kSearchStages * kTileBytes, "selection arrays fit in the ring");
   __shared__ DecSearchShared sh;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
-  const int n = static_cast<int>(blockIdx.x) / H, h = static_cast<int>(blockIdx.x) % H;
+  const int SC = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const long long row = blockIdx.y;
+  const int n = static_cast<int>(row / H), h = static_cast<int>(row % H);
   const int kvh = h / (H / Hkv);
-  const long long row = static_cast<long long>(n) * H + h;
   int32_t* out = idx + row * Nbm;
   uint32_t* obits = bits + row * W;
+  if (c == 0 && row == 0) block_count_prefix(lens, N, Lmax, B, rowstart, sh.ubuf);
   const int len = __ldg(lens + n);
-  if (len < 1 || len > Lmax) {   // not a cache length this call can serve: nothing selected
-    if (tid == 0) {
-      count[row] = 0;
-      atomicCAS(status, 0u, kStatusLenCode | (static_cast<unsigned>(n < (1 << 24) ? n : (1 << 24) - 1) << 8));
+  if (len < 1 || len > Lmax) {   // not a cache length this call can serve: nothing selected, zero output
+    if (c == 0) {
+      for (int k = tid; k < D; k += kDecThreads) o[row * D + k] = __float2bfloat16(0.f);
+      if (tid == 0) {
+        count[row] = 0;
+        atomicCAS(status, 0u, kStatusLenCode | (static_cast<unsigned>(n < (1 << 24) ? n : (1 << 24) - 1) << 8));
+      }
+      for (int w = tid; w < W; w += kDecThreads) obits[w] = 0u;
     }
-    for (int w = tid; w < W; w += kDecThreads) obits[w] = 0u;
     return;
   }
   const int t = len - 1, Jt = t / B, nb = Jt + 1, off = h % S, r = B / S;
   const int ns = t >= off ? (t - off) / S + 1 : 0;   // sampled keys at or before t
   const int nt = (ns + kSearchTile - 1) / kSearchTile;
+  const int i0 = c * tpc, i1 = min(i0 + tpc, nt);      // this CTA's tiles
+  const int bpc = tpc * (kSearchTile / r);
+  const int J0 = min(c * bpc, nb), J1 = min(J0 + bpc, nb);   // and key blocks
   if (tid == 0) {
     for (int st = 0; st < kSearchStages; ++st) mbar_init(smem_u32(&sh.full[st]), 1);
     sh.abort = 0;
     fence_mbar_init();
   }
-  // lanes 2k and 2k+1 score key k of a tile, each over half of d; the half of
-  // q they need stays in registers
-  const int kr = tid >> 1, half = tid & 1;
-  float qr[D / 2];
+  // warp w scores keys 16w .. 16w + 15 of a tile on m16n8k16 tiles: the keys
+  // are A fragments (ldmatrix from the swizzled tile), q is column 0 of the B
+  // fragments (the other seven columns are zero)
+  const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+  const int mi = lane >> 3, ri = lane & 7;
+  uint32_t qb[D / 16][2];
 #pragma unroll
-  for (int c = 0; c < D / 2; c += 2) {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + row * D + half * (D / 2) + c));
-    qr[c] = f.x * sl2;
-    qr[c + 1] = f.y * sl2;
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const __nv_bfloat16* qr = q + row * D + 16 * ks + 2 * tig;
+    qb[ks][0] = gid == 0 ? __ldg(reinterpret_cast<const uint32_t*>(qr)) : 0u;
+    qb[ks][1] = gid == 0 ? __ldg(reinterpret_cast<const uint32_t*>(qr + 8)) : 0u;
   }
   __syncthreads();
   const Guard guard{&sh.abort, status, limit_ns};
   // tile i: the sampled keys of strides 128 i .. 128 i + 127 of sequence n
   auto issue = [&](int i) {
-    const int st = i % kSearchStages;
+    const int st = (i - i0) % kSearchStages;
     const uint32_t fb = smem_u32(&sh.full[st]);
     mbar_expect_tx(fb, kTileBytes);
     uint8_t* dst = smem + st * kTileBytes;
@@ -263,72 +344,88 @@ __global__ void __launch_bounds__(kDecThreads) decode_search_kernel(
       tma_load_4d(smem_u32(dst + a * kSearchTile * 128), &mks, fb, a * 64, kvh, off,
                   n * (Lmax / S) + i * kSearchTile);
   };
-  int issued = 0;
-  if (tid == 0) {
+  int issued = i0;
+  if (tid == 0 && i0 < i1) {
     tma_prefetch_desc(&mks);
-    for (; issued < nt && issued < kSearchStages; ++issued) issue(issued);
+    for (; issued < i1 && issued < i0 + kSearchStages; ++issued) issue(issued);
   }
   // scores (log2 units) of the sampled keys, to the workspace row
   float* sc = scores + row * Ns_max;
   float lmax = -INFINITY;
   bool ok = true;
-  for (int i = 0; i < nt; ++i) {
-    const int st = i % kSearchStages;
-    if (!wait_bar(smem_u32(&sh.full[st]), (i / kSearchStages) & 1, guard, 1)) ok = false;
+  for (int i = i0; i < i1; ++i) {
+    const int st = (i - i0) % kSearchStages;
+    if (!wait_bar(smem_u32(&sh.full[st]), ((i - i0) / kSearchStages) & 1, guard, 1)) ok = false;
     if (!__syncthreads_and(ok)) break;
-    const uint8_t* tile = smem + st * kTileBytes;
-    float acc0 = 0.f, acc1 = 0.f;
+    const uint32_t tile = smem_u32(smem + st * kTileBytes);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < D / 2; c += 8) {
-      const uint4 v4 = *reinterpret_cast<const uint4*>(tile + swz128(kr, half * (D / 2) + c));
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(p2[e]);
-        acc0 = fmaf(f.x, qr[c + 2 * e], acc0);
-        acc1 = fmaf(f.y, qr[c + 2 * e + 1], acc1);
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t a[4];
+      ldsm_x4(tile + swz<kSearchTile>(16 * warp + (mi & 1) * 8 + ri, 16 * ks + (mi >> 1) * 8), a);
+      mma_bf16(acc, a, qb[ks][0], qb[ks][1]);
+    }
+    if (tig == 0) {   // column 0: keys 16w + gid (acc 0) and 16w + gid + 8 (acc 2)
+      const int j = i * kSearchTile + 16 * warp + gid;
+      if (j < ns) {
+        sc[j] = acc[0] * sl2;
+        lmax = fmaxf(lmax, acc[0] * sl2);
+      }
+      if (j + 8 < ns) {
+        sc[j + 8] = acc[2] * sl2;
+        lmax = fmaxf(lmax, acc[2] * sl2);
       }
     }
-    float sv = acc0 + acc1;
-    sv += __shfl_xor_sync(0xffffffffu, sv, 1);
-    const int j = i * kSearchTile + kr;
-    if (j < ns) {
-      if (half == 0) sc[j] = sv;
-      lmax = fmaxf(lmax, sv);
-    }
     __syncthreads();   // stage st is free again
-    if (tid == 0 && issued < nt) issue(issued++);
+    if (tid == 0 && issued < i1) issue(issued++);
   }
   if (tid == 0) {
-    for (int i = (issued > kSearchStages ? issued - kSearchStages : 0); i < issued; ++i)
-      drain_bar(smem_u32(&sh.full[i % kSearchStages]), (i / kSearchStages) & 1, kDrainLimitNs);
+    for (int i = (issued - i0 > kSearchStages ? issued - kSearchStages : i0); i < issued; ++i)
+      drain_bar(smem_u32(&sh.full[(i - i0) % kSearchStages]), ((i - i0) / kSearchStages) & 1, kDrainLimitNs);
   }
-  if (!__syncthreads_and(ok)) {   // a wait ran out (status recorded): nothing selected
-    if (tid == 0) count[row] = 0;
-    for (int w = tid; w < W; w += kDecThreads) obits[w] = 0u;
-    return;
-  }
-  const float mx = block_max(lmax, sh.fbuf);
+  // a wait that ran out (status recorded) leaves this run without mass
+  const bool good = __syncthreads_and(ok);
+  const float cm = good ? block_max(lmax, sh.fbuf) : -INFINITY;
   __syncthreads();   // the scores of other threads are visible (global writes, same block)
-  // block mass: exp2 of the scores summed over the r strides of each block
-  for (int J = tid; J < nb; J += kDecThreads) {
+  // this run's block masses on its own max: exp2 of the scores summed over the r
+  // strides of each block
+  float* mrow = mass + row * Nbm;
+  for (int J = J0 + tid; J < J1; J += kDecThreads) {
     float m = 0.f;
-    const int j1 = min((J + 1) * r, ns);
-    for (int j = J * r; j < j1; ++j) m += exp2f(sc[j] - mx);
-    sh.mass[J] = m;
+    if (cm > -INFINITY) {
+      const int j1 = min((J + 1) * r, ns);
+      for (int j = J * r; j < j1; ++j) m += exp2f(sc[j] - cm);
+    }
+    mrow[J] = m;
+  }
+  if (tid == 0) cmax[row * SC + c] = cm;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(arrive + row, 1u) == static_cast<unsigned>(SC - 1);
+  __syncthreads();
+  if (!sh.last) return;
+  __threadfence();
+  // the last CTA of the row: every run's masses on the row max, in the ring's
+  // shared memory (every copy has landed)
+  float* smass = reinterpret_cast<float*>(smem);
+  uint32_t* swbits = reinterpret_cast<uint32_t*>(smem + kMaxBlocks * 4);
+  float M = -INFINITY;
+  for (int k = 0; k < SC; ++k) M = fmaxf(M, __ldcg(cmax + row * SC + k));
+  for (int J = tid; J < nb; J += kDecThreads) {
+    const float ck = __ldcg(cmax + row * SC + J / bpc);
+    smass[J] = ck > -INFINITY ? __ldcg(mrow + J) * exp2f(ck - M) : 0.f;
   }
   __syncthreads();
 
-  if (group_mass) {   // one mask per GQA group: the head's masses, normalised, for the group kernel
+  if (group) {   // one mask per GQA group: the head's masses, normalised, for the group kernel
     float lsum = 0.f;
-    for (int J = tid; J < nb; J += kDecThreads) lsum += sh.mass[J];
+    for (int J = tid; J < nb; J += kDecThreads) lsum += smass[J];
     const float tot = block_sum<float>(lsum, sh.fbuf);
     const float inv = tot > 0.f ? 1.0f / tot : 0.f;
-    float* mrow = group_mass + row * Nbm;
-    for (int J = tid; J < nb; J += kDecThreads) mrow[J] = sh.mass[J] * inv;
+    for (int J = tid; J < nb; J += kDecThreads) mrow[J] = smass[J] * inv;
     return;
   }
-  block_select(sh, nb, Jt, tau, out, Nbm, obits, W, count + row, 1);
+  block_select(sh, smass, swbits, nb, Jt, tau, out, Nbm, obits, W, count + row, 1);
 }
 
 // One mask per GQA group (decode): the block masses of the group's g heads,
@@ -341,6 +438,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_select_kernel(const 
                                                                          int32_t* __restrict__ idx,
                                                                          uint32_t* __restrict__ bits, int Nbm, int W) {
   __shared__ DecSearchShared sh;
+  __shared__ float smass[kMaxBlocks];
+  __shared__ uint32_t swbits[kMaxBlocks / 32];
   const int tid = threadIdx.x;
   const int n = static_cast<int>(blockIdx.x) / Hkv, kvh = static_cast<int>(blockIdx.x) % Hkv;
   const int g = H / Hkv;
@@ -355,307 +454,441 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_select_kernel(const 
   for (int J = tid; J < nb; J += kDecThreads) {
     float m = 0.f;
     for (int r = 0; r < g; ++r) m += group_mass[(row0 + r) * Nbm + J];
-    sh.mass[J] = m;
+    smass[J] = m;
   }
   __syncthreads();
-  block_select(sh, nb, Jt, tau, idx + row0 * Nbm, Nbm, bits + row0 * W, W, count + row0, g);
+  block_select(sh, smass, swbits, nb, Jt, tau, idx + row0 * Nbm, Nbm, bits + row0 * W, W, count + row0, g);
 }
 
 // ------------------------------------------------------------------ attention
-constexpr int kDecChunk = 16;   // key blocks per attention CTA (half a bitmap word)
 constexpr int kDecStages = 3;
 
 template <int BN, int D>
 struct DecAttnCfg {
   static constexpr int kTileBytes = BN * D * 2;
   static constexpr int kStageBytes = 2 * kTileBytes;   // K and V
-  static constexpr int kSmem = kDecStages * kStageBytes + 1024;
-  static_assert(kDecWarps * 8 * D * 4 <= kStageBytes, "the warp partials fit in one stage");
+  static constexpr int kMergeLd = D / 2 + 4;            // merge rows: half of d, padded against bank conflicts
+  static constexpr int kMergeBytes = (BN / 16) * 8 * kMergeLd * 4;
+  static constexpr int kSmem = kDecStages * kStageBytes + kMergeBytes + 1024;
 };
 
 struct DecAttnCtrl {
   uint64_t full[kDecStages];
   int abort;
-  uint32_t hbits[8];
+  int last;                                // this CTA completes the current row
+  int clo, chi;                            // the CTAs whose shares meet the current row
   float2 ml[kDecWarps][8];                 // warp partials: (max, sum) per head
   __nv_bfloat16 p[kDecWarps][8][24];       // per warp: P of its 16 keys, [head][key] (rows padded)
 };
 
-// Position of the (i+1)-th set bit of `set` (i < popcount).
-__device__ __forceinline__ int nth_bit(uint32_t set, int i) {
-  for (int k = 0; k < i; ++k) set &= set - 1u;
-  return __ffs(static_cast<int>(set)) - 1;
+// The rows of one attention CTA's share [b0, b1) of the flattened space in which
+// row (n, kvh) holds the causal key blocks 0 .. nbl_n - 1 of sequence n, rows
+// n-major then kv head; rowstart is the exclusive prefix of nbl_n (a sequence
+// of length outside [1, Lmax] has none).  A segment is the part [Ja, Jb) of one
+// row inside the share.
+struct SegWalk {
+  const int32_t* rs;
+  int Hkv;
+  long long pos, b1;
+  int n, kvh, Ja, Jb;
+  __device__ __forceinline__ void load() {
+    const long long base = static_cast<long long>(Hkv) * __ldg(rs + n);
+    const int nbl = __ldg(rs + n + 1) - __ldg(rs + n);
+    const long long o = pos - base;
+    kvh = static_cast<int>(o / nbl);
+    Ja = static_cast<int>(o % nbl);
+    const long long rend = base + static_cast<long long>(kvh + 1) * nbl;
+    Jb = Ja + static_cast<int>((b1 < rend ? b1 : rend) - pos);
+  }
+  __device__ bool begin(const int32_t* rs_, int N, int Hkv_, long long b0, long long b1_) {
+    rs = rs_;
+    Hkv = Hkv_;
+    pos = b0;
+    b1 = b1_;
+    if (pos >= b1) return false;
+    // the last sequence whose rows start at or before b0 (it has blocks: b0 < total)
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (static_cast<long long>(Hkv) * __ldg(rs + mid) <= pos) lo = mid;
+      else hi = mid - 1;
+    }
+    n = lo;
+    load();
+    return true;
+  }
+  __device__ bool next() {
+    pos += Jb - Ja;
+    if (pos >= b1) return false;
+    if (pos == static_cast<long long>(Hkv) * __ldg(rs + n + 1)) {   // the next sequence with blocks
+      do ++n;
+      while (__ldg(rs + n + 1) == __ldg(rs + n));
+    }
+    load();
+    return true;
+  }
+};
+
+// Bits of word w of a segment's blocks, and the union of the group's kept bits there.
+__device__ __forceinline__ uint32_t seg_mask(const SegWalk& s, int w) {
+  const int lo = max(s.Ja - 32 * w, 0), hi = min(s.Jb - 32 * w, 32);
+  const uint32_t upto = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+  return upto & ~((1u << lo) - 1u);
+}
+__device__ __forceinline__ uint32_t group_word(const uint32_t* __restrict__ bits, const SegWalk& s, int H, int g,
+                                               int W, int w) {
+  const uint32_t* b = bits + (static_cast<long long>(s.n) * H + s.kvh * g) * W + w;
+  uint32_t u = 0u;
+  for (int hh = 0; hh < g; ++hh) u |= __ldg(b + static_cast<long long>(hh) * W);
+  return u & seg_mask(s, w);
 }
 
-// Byte offset of element (row, c) in a TMA tile of rows x D bf16 stored as D/64
-// column blocks of rows x 128 bytes with the 128-byte swizzle (c a multiple of 8
-// when used as a 16-byte row address).
-template <int BN>
-__device__ __forceinline__ uint32_t swz(int row, int c) {
-  return static_cast<uint32_t>((c >> 6) * (BN * 128) + row * 128 + ((((c & 63) >> 3) ^ (row & 7)) << 4) + (c & 7) * 2);
+// The kept blocks of a CTA's share in order (the copy side's walk).
+struct KeptWalk {
+  SegWalk s;
+  bool live;
+  int w;
+  uint32_t rem;
+  __device__ void begin(const int32_t* rs, int N, int Hkv, long long b0, long long b1, const uint32_t* bits, int H,
+                        int g, int W) {
+    live = s.begin(rs, N, Hkv, b0, b1);
+    if (live) {
+      w = s.Ja >> 5;
+      rem = group_word(bits, s, H, g, W, w);
+    }
+  }
+  __device__ bool next(const uint32_t* bits, int H, int g, int W, int& n, int& J) {
+    while (live) {
+      if (rem) {
+        J = 32 * w + __ffs(static_cast<int>(rem)) - 1;
+        rem &= rem - 1u;
+        n = s.n;
+        return true;
+      }
+      if (++w <= (s.Jb - 1) >> 5) {
+        rem = group_word(bits, s, H, g, W, w);
+        continue;
+      }
+      live = s.next();
+      if (live) {
+        w = s.Ja >> 5;
+        rem = group_word(bits, s, H, g, W, w);
+      }
+    }
+    return false;
+  }
+};
+
+// owner(x): the CTA whose share [c T / P, (c+1) T / P) holds flattened block x.
+__device__ __forceinline__ int share_owner(long long x, long long T, int P) {
+  return static_cast<int>(((x + 1) * P - 1) / T);
+}
+__device__ __forceinline__ long long share_start(int c, long long T, int P) {
+  return static_cast<long long>(c) * T / P;
 }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col).
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// One CTA per (sequence n, kv head, 16 key blocks).  Each kept block J comes in
-// once for the whole GQA group; the group's heads are the 8 columns of
-// m16n8k16 tiles (heads beyond the group and heads that did not keep J are
-// masked).  Warp w owns keys 16w..16w+15 of every block and keeps its own
-// online softmax and O^T over them (a split over keys inside the CTA):
+// grid P (one CTA per SM): CTA c walks its share [c T / P, (c+1) T / P) of the
+// flattened (sequence, kv head, causal block) space, T = Hkv * rowstart[N].  Each
+// kept block J of a row comes in once for the whole GQA group; the group's heads
+// are the 8 columns of m16n8k16 tiles (heads beyond the group and heads that did
+// not keep J are masked).  Warp w owns keys 16w..16w+15 of every block and keeps
+// its own online softmax and O^T over them (a split over keys inside the CTA):
 //   S^T [16 keys x heads] = K_J [16 keys x d] . Q^T [d x heads]
 //   per head: running max and sum over the warp's keys, P (bf16) re-laid from
 //   the accumulator fragment to the operand fragment through a small per-warp
 //   buffer
 //   O^T [d x heads] += V_J^T [d x 16 keys] . P^T [16 keys x heads]
-// No cross-warp exchange per block: one barrier frees the stage.  At the end the
-// eight warp partials are merged into the chunk's partial.  Q^T stays in
-// registers as B fragments; K comes in as A fragments by ldmatrix, V^T by
-// ldmatrix.trans, both from the 128-byte swizzled TMA tiles.
+// No cross-warp exchange per block: one barrier frees the stage.  At the end of
+// each row segment the warp partials merge into the CTA's partial for the row,
+// slot (row + c) of the workspace (row n Hkv + kvh; the slots of the (row, CTA)
+// pairs that exist are distinct because rows and shares are both in order).
+// Q^T stays in registers as B fragments; K comes in as A fragments by ldmatrix,
+// V^T by ldmatrix.trans, both from the 128-byte swizzled TMA tiles.  The copies
+// run ahead across rows.
 template <int BN, int D>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
     const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
-    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lens, const uint32_t* __restrict__ bits,
-    int Lmax, int H, int Hkv, int W, int NC, float sl2, float* __restrict__ part, unsigned int* status,
-    uint64_t limit_ns) {
+    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lens, const int32_t* __restrict__ rowstart,
+    const uint32_t* __restrict__ bits, int N, int Lmax, int H, int Hkv, int W, float sl2, float* __restrict__ part,
+    unsigned int* __restrict__ row_arrive, __nv_bfloat16* __restrict__ o, unsigned int* status, uint64_t limit_ns) {
   using C = DecAttnCfg<BN, D>;
   constexpr int kKeyWarps = BN / 16;  // warps that own keys (8 at B = 128, 4 at B = 64)
   constexpr int kDSteps = D / 16;     // k-steps of S (over d)
   constexpr int kOTiles = D / 16;     // d-row tiles of O^T
+  constexpr int kLd = C::kMergeLd;
   __shared__ DecAttnCtrl ctl;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* ow = reinterpret_cast<float*>(smem + kDecStages * C::kStageBytes);   // merge rows [warp][head][kLd]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;   // mma fragment coordinates
-  const int chunk = static_cast<int>(blockIdx.x), kvh = static_cast<int>(blockIdx.y), n = static_cast<int>(blockIdx.z);
+  const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   const int g = H / Hkv;
-  const int len = __ldg(lens + n);
-  const int t = len - 1;
-  const int J0 = chunk * kDecChunk;
-  const bool live = len >= 1 && len <= Lmax && J0 <= t / BN;
-  if (tid < 8) {
-    uint32_t b = 0u;
-    if (live && tid < g) b = __ldg(bits + (static_cast<long long>(n) * H + kvh * g + tid) * W + (J0 >> 5));
-    ctl.hbits[tid] = (b >> (J0 & 31)) & ((1u << kDecChunk) - 1u);
-  }
+  const long long T = static_cast<long long>(Hkv) * __ldg(rowstart + N);
+  const long long b0 = share_start(c, T, P), b1 = share_start(c + 1, T, P);
+  if (b0 >= b1) return;
   if (tid == 0) {
-    for (int s = 0; s < kDecStages; ++s) mbar_init(smem_u32(&ctl.full[s]), 1);
+    for (int st = 0; st < kDecStages; ++st) mbar_init(smem_u32(&ctl.full[st]), 1);
     ctl.abort = 0;
     fence_mbar_init();
   }
-  // Q^T as B fragments: b0 = Q[head gid][16 ks + 2 tig, +1], b1 = the same at +8
-  uint32_t qb[kDSteps][2];
-  {
-    const bool hv = gid < g;
-    const __nv_bfloat16* qr = q + (static_cast<long long>(n) * H + kvh * g + (hv ? gid : 0)) * D;
-#pragma unroll
-    for (int ks = 0; ks < kDSteps; ++ks) {
-      qb[ks][0] = hv ? __ldg(reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * tig)) : 0u;
-      qb[ks][1] = hv ? __ldg(reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * tig + 8)) : 0u;
-    }
-  }
   __syncthreads();
-  uint32_t any = 0;
-  for (int hh = 0; hh < g; ++hh) any |= ctl.hbits[hh];
   const Guard guard{&ctl.abort, status, limit_ns};
 
-  // the chunk's kept blocks, ascending; block i of the sequence goes to stage i % kDecStages
-  auto issue = [&](int i) {
-    const int J = J0 + nth_bit(any, i);
-    const int st = i % kDecStages;
+  // kept block number i of the share goes to stage i % kDecStages
+  KeptWalk pk;   // thread 0's walk: the copies
+  int issued = 0;
+  auto issue_next = [&]() {
+    int nn, J;
+    if (!pk.next(bits, H, g, W, nn, J)) return;
+    const int st = issued % kDecStages;
     const uint32_t fb = smem_u32(&ctl.full[st]);
     mbar_expect_tx(fb, C::kStageBytes);
     uint8_t* dst = smem + st * C::kStageBytes;
-    const int r0 = n * Lmax + J * BN;
+    const int r0 = nn * Lmax + J * BN;
     for (int a = 0; a < D / 64; ++a) {
-      tma_load_3d(smem_u32(dst + a * BN * 128), &mk, fb, a * 64, kvh, r0);
-      tma_load_3d(smem_u32(dst + C::kTileBytes + a * BN * 128), &mv, fb, a * 64, kvh, r0);
+      tma_load_3d(smem_u32(dst + a * BN * 128), &mk, fb, a * 64, pk.s.kvh, r0);
+      tma_load_3d(smem_u32(dst + C::kTileBytes + a * BN * 128), &mv, fb, a * 64, pk.s.kvh, r0);
     }
+    ++issued;
   };
-  const int n_blk = __popc(any);
-  int issued = 0;   // thread 0: copies issued so far
   if (tid == 0) {
     tma_prefetch_desc(&mk);
     tma_prefetch_desc(&mv);
-    for (; issued < n_blk && issued < kDecStages; ++issued) issue(issued);
+    pk.begin(rowstart, N, Hkv, b0, b1, bits, H, g, W);
+    for (int i = 0; i < kDecStages; ++i) issue_next();
   }
 
-  // This warp's running max and sum for the lane's two head columns (2 tig,
-  // 2 tig + 1), and its O^T tiles (d rows 16 mt + gid and + 8, the same columns).
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-  float o_acc[kOTiles][4];
-#pragma unroll
-  for (int mt = 0; mt < kOTiles; ++mt)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) o_acc[mt][c] = 0.f;
   const int mi = lane >> 3, ri = lane & 7;   // ldmatrix: this lane's matrix and row
   bool ok = true;
-  for (int i = 0; i < n_blk; ++i) {
-    const int J = J0 + nth_bit(any, i);
-    const uint32_t jb = 1u << (J - J0);
-    const int st = i % kDecStages;
-    if (!wait_bar(smem_u32(&ctl.full[st]), (i / kDecStages) & 1, guard, 1)) ok = false;
-    if (!__syncthreads_and(ok)) break;
-    if (warp < kKeyWarps) {
-      const uint32_t ks_base = smem_u32(smem + st * C::kStageBytes);
-      const uint32_t vs_base = ks_base + C::kTileBytes;
-      const bool keep0 = 2 * tig < g && (ctl.hbits[2 * tig] & jb);
-      const bool keep1 = 2 * tig + 1 < g && (ctl.hbits[2 * tig + 1] & jb);
-      // S^T tile: keys 16w + gid (acc 0, 1) and 16w + gid + 8 (acc 2, 3)
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int seq = 0;   // kept blocks consumed
+  SegWalk cs;
+  bool more = cs.begin(rowstart, N, Hkv, b0, b1);
+  while (more) {
+    const int n = cs.n, kvh = cs.kvh;
+    const int t = __ldg(lens + n) - 1;
+    // Q^T as B fragments: b0 = Q[head gid][16 ks + 2 tig, +1], b1 = the same at +8
+    uint32_t qb[kDSteps][2];
+    {
+      const bool hv = gid < g;
+      const __nv_bfloat16* qr = q + (static_cast<long long>(n) * H + kvh * g + (hv ? gid : 0)) * D;
 #pragma unroll
       for (int ks = 0; ks < kDSteps; ++ks) {
-        uint32_t a[4];
-        ldsm_x4(ks_base + swz<BN>(16 * warp + (mi & 1) * 8 + ri, 16 * ks + (mi >> 1) * 8), a);
-        mma_bf16(acc, a, qb[ks][0], qb[ks][1]);
-      }
-      const int key0 = J * BN + 16 * warp + gid;
-      const bool v0 = key0 <= t, v1 = key0 + 8 <= t;
-      const float s0 = (keep0 && v0) ? acc[0] * sl2 : -INFINITY;
-      const float s1 = (keep1 && v0) ? acc[1] * sl2 : -INFINITY;
-      const float s2 = (keep0 && v1) ? acc[2] * sl2 : -INFINITY;
-      const float s3 = (keep1 && v1) ? acc[3] * sl2 : -INFINITY;
-      // per head column: max over the warp's 16 keys
-      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-#pragma unroll
-      for (int x = 4; x < 32; x <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, x));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, x));
-      }
-      const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-      // a column with nothing so far and nothing now keeps alpha 1 (its O is 0)
-      const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m_run[0] - mn0);
-      const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m_run[1] - mn1);
-      const __nv_bfloat16 p0 = __float2bfloat16(s0 == -INFINITY ? 0.f : exp2f(s0 - mn0));
-      const __nv_bfloat16 p1 = __float2bfloat16(s1 == -INFINITY ? 0.f : exp2f(s1 - mn1));
-      const __nv_bfloat16 p2 = __float2bfloat16(s2 == -INFINITY ? 0.f : exp2f(s2 - mn0));
-      const __nv_bfloat16 p3 = __float2bfloat16(s3 == -INFINITY ? 0.f : exp2f(s3 - mn1));
-      // sums of the bf16 P that P V uses
-      float sm0 = __bfloat162float(p0) + __bfloat162float(p2), sm1 = __bfloat162float(p1) + __bfloat162float(p3);
-#pragma unroll
-      for (int x = 4; x < 32; x <<= 1) {
-        sm0 += __shfl_xor_sync(0xffffffffu, sm0, x);
-        sm1 += __shfl_xor_sync(0xffffffffu, sm1, x);
-      }
-      l_run[0] = l_run[0] * al0 + sm0;
-      l_run[1] = l_run[1] * al1 + sm1;
-      m_run[0] = mn0;
-      m_run[1] = mn1;
-      // P from the accumulator layout (key rows, head columns) to the operand
-      // layout (b0 = P[head gid][keys 2 tig, +1], b1 = keys + 8)
-      __nv_bfloat16(*pw)[24] = ctl.p[warp];
-      pw[2 * tig][gid] = p0;
-      pw[2 * tig + 1][gid] = p1;
-      pw[2 * tig][gid + 8] = p2;
-      pw[2 * tig + 1][gid + 8] = p3;
-      __syncwarp();
-      const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&pw[gid][2 * tig]);
-      const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&pw[gid][2 * tig + 8]);
-      __syncwarp();
-#pragma unroll
-      for (int mt = 0; mt < kOTiles; ++mt) {
-        o_acc[mt][0] *= al0;
-        o_acc[mt][1] *= al1;
-        o_acc[mt][2] *= al0;
-        o_acc[mt][3] *= al1;
-        uint32_t a[4];
-        ldsm_x4_t(vs_base + swz<BN>(16 * warp + (mi >> 1) * 8 + ri, 16 * mt + (mi & 1) * 8), a);
-        mma_bf16(o_acc[mt], a, b0, b1);
+        qb[ks][0] = hv ? __ldg(reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * tig)) : 0u;
+        qb[ks][1] = hv ? __ldg(reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * tig + 8)) : 0u;
       }
     }
-    __syncthreads();   // stage st is free again
-    if (tid == 0 && issued < n_blk) issue(issued++);
-  }
-  // in-flight copies land before the CTA exits (only after an abort can any be left)
-  if (tid == 0) {
-    for (int i = (issued > kDecStages ? issued - kDecStages : 0); i < issued; ++i)
-      drain_bar(smem_u32(&ctl.full[i % kDecStages]), (i / kDecStages) & 1, kDrainLimitNs);
-  }
-  const bool done = __syncthreads_and(ok) && live;
-  // merge the warp partials: stage 0 holds each warp's O^T as [warp][head][d] fp32
-  float* ow = reinterpret_cast<float*>(smem);
-  if (warp < kKeyWarps) {
-    if (gid == 0) {
+    // This warp's running max and sum for the lane's two head columns (2 tig,
+    // 2 tig + 1), and its O^T tiles (d rows 16 mt + gid and + 8, the same columns).
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    float o_acc[kOTiles][4];
+#pragma unroll
+    for (int mt = 0; mt < kOTiles; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o_acc[mt][e] = 0.f;
+    const uint32_t* hrow = bits + (static_cast<long long>(n) * H + kvh * g) * W;
+    for (int w = cs.Ja >> 5; ok && w <= (cs.Jb - 1) >> 5; ++w) {
+      // the lane's two heads' kept bits in this word, and the group's union
+      const uint32_t hb0 = 2 * tig < g ? __ldg(hrow + static_cast<long long>(2 * tig) * W + w) : 0u;
+      const uint32_t hb1 = 2 * tig + 1 < g ? __ldg(hrow + static_cast<long long>(2 * tig + 1) * W + w) : 0u;
+      uint32_t rem = group_word(bits, cs, H, g, W, w);
+      while (rem) {
+        const int jw = __ffs(static_cast<int>(rem)) - 1;
+        rem &= rem - 1u;
+        const int J = 32 * w + jw;
+        const int st = seq % kDecStages;
+        if (!wait_bar(smem_u32(&ctl.full[st]), (seq / kDecStages) & 1, guard, 1)) ok = false;
+        if (!__syncthreads_and(ok)) {
+          ok = false;
+          break;
+        }
+        if (warp < kKeyWarps) {
+          const uint32_t ks_base = smem_u32(smem + st * C::kStageBytes);
+          const uint32_t vs_base = ks_base + C::kTileBytes;
+          const bool keep0 = (hb0 >> jw) & 1u, keep1 = (hb1 >> jw) & 1u;
+          // S^T tile: keys 16w + gid (acc 0, 1) and 16w + gid + 8 (acc 2, 3)
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < kDSteps; ++ks) {
+            uint32_t a[4];
+            ldsm_x4(ks_base + swz<BN>(16 * warp + (mi & 1) * 8 + ri, 16 * ks + (mi >> 1) * 8), a);
+            mma_bf16(acc, a, qb[ks][0], qb[ks][1]);
+          }
+          const int key0 = J * BN + 16 * warp + gid;
+          const bool v0 = key0 <= t, v1 = key0 + 8 <= t;
+          const float s0 = (keep0 && v0) ? acc[0] * sl2 : -INFINITY;
+          const float s1 = (keep1 && v0) ? acc[1] * sl2 : -INFINITY;
+          const float s2 = (keep0 && v1) ? acc[2] * sl2 : -INFINITY;
+          const float s3 = (keep1 && v1) ? acc[3] * sl2 : -INFINITY;
+          // per head column: max over the warp's 16 keys
+          float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+          for (int x = 4; x < 32; x <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, x));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, x));
+          }
+          const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+          // a column with nothing so far and nothing now keeps alpha 1 (its O is 0)
+          const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m_run[0] - mn0);
+          const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m_run[1] - mn1);
+          const __nv_bfloat16 p0 = __float2bfloat16(s0 == -INFINITY ? 0.f : exp2f(s0 - mn0));
+          const __nv_bfloat16 p1 = __float2bfloat16(s1 == -INFINITY ? 0.f : exp2f(s1 - mn1));
+          const __nv_bfloat16 p2 = __float2bfloat16(s2 == -INFINITY ? 0.f : exp2f(s2 - mn0));
+          const __nv_bfloat16 p3 = __float2bfloat16(s3 == -INFINITY ? 0.f : exp2f(s3 - mn1));
+          // sums of the bf16 P that P V uses
+          float sm0 = __bfloat162float(p0) + __bfloat162float(p2), sm1 = __bfloat162float(p1) + __bfloat162float(p3);
+#pragma unroll
+          for (int x = 4; x < 32; x <<= 1) {
+            sm0 += __shfl_xor_sync(0xffffffffu, sm0, x);
+            sm1 += __shfl_xor_sync(0xffffffffu, sm1, x);
+          }
+          l_run[0] = l_run[0] * al0 + sm0;
+          l_run[1] = l_run[1] * al1 + sm1;
+          m_run[0] = mn0;
+          m_run[1] = mn1;
+          // P from the accumulator layout (key rows, head columns) to the operand
+          // layout (b0 = P[head gid][keys 2 tig, +1], b1 = keys + 8)
+          __nv_bfloat16(*pw)[24] = ctl.p[warp];
+          pw[2 * tig][gid] = p0;
+          pw[2 * tig + 1][gid] = p1;
+          pw[2 * tig][gid + 8] = p2;
+          pw[2 * tig + 1][gid + 8] = p3;
+          __syncwarp();
+          const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(&pw[gid][2 * tig]);
+          const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(&pw[gid][2 * tig + 8]);
+          __syncwarp();
+#pragma unroll
+          for (int mt = 0; mt < kOTiles; ++mt) {
+            o_acc[mt][0] *= al0;
+            o_acc[mt][1] *= al1;
+            o_acc[mt][2] *= al0;
+            o_acc[mt][3] *= al1;
+            uint32_t a[4];
+            ldsm_x4_t(vs_base + swz<BN>(16 * warp + (mi >> 1) * 8 + ri, 16 * mt + (mi & 1) * 8), a);
+            mma_bf16(o_acc[mt], a, pb0, pb1);
+          }
+        }
+        __syncthreads();   // stage st is free again
+        if (tid == 0) issue_next();
+        ++seq;
+      }
+    }
+    // the row's partial from this CTA: the warp partials merged (nothing after a
+    // wait that ran out)
+    const long long prow = (static_cast<long long>(n) * Hkv + kvh + c) * g;
+    if (warp < kKeyWarps && gid == 0) {
       ctl.ml[warp][2 * tig] = make_float2(m_run[0], l_run[0]);
       ctl.ml[warp][2 * tig + 1] = make_float2(m_run[1], l_run[1]);
     }
+    __syncthreads();
+    const int hh = warp;   // one warp per head of the group
+    float f[kKeyWarps];
+    bool has = false;
+    if (hh < g) {
+      float Mx = -INFINITY;
 #pragma unroll
-    for (int mt = 0; mt < kOTiles; ++mt) {
-      const int d0 = 16 * mt + gid;
-      ow[(warp * 8 + 2 * tig) * D + d0] = o_acc[mt][0];
-      ow[(warp * 8 + 2 * tig + 1) * D + d0] = o_acc[mt][1];
-      ow[(warp * 8 + 2 * tig) * D + d0 + 8] = o_acc[mt][2];
-      ow[(warp * 8 + 2 * tig + 1) * D + d0 + 8] = o_acc[mt][3];
+      for (int w = 0; w < kKeyWarps; ++w) Mx = fmaxf(Mx, ctl.ml[w][hh].x);
+      has = ok && Mx > -INFINITY;
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kKeyWarps; ++w) {
+        const float2 ml = ctl.ml[w][hh];
+        f[w] = (has && ml.x > -INFINITY) ? exp2f(ml.x - Mx) : 0.f;
+        L += ml.y * f[w];
+      }
+      if (lane == 0) {
+        part[(prow + hh) * (D + 2)] = has ? Mx : -INFINITY;
+        part[(prow + hh) * (D + 2) + 1] = has ? L : 0.f;
+      }
     }
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {   // the two halves of d in turn through the merge rows
+      if (warp < kKeyWarps) {
+#pragma unroll
+        for (int mt = hf * kOTiles / 2; mt < (hf + 1) * kOTiles / 2; ++mt) {
+          const int d0 = 16 * mt + gid - hf * (D / 2);
+          ow[(warp * 8 + 2 * tig) * kLd + d0] = o_acc[mt][0];
+          ow[(warp * 8 + 2 * tig + 1) * kLd + d0] = o_acc[mt][1];
+          ow[(warp * 8 + 2 * tig) * kLd + d0 + 8] = o_acc[mt][2];
+          ow[(warp * 8 + 2 * tig + 1) * kLd + d0 + 8] = o_acc[mt][3];
+        }
+      }
+      __syncthreads();
+      if (hh < g) {
+        for (int d = lane; d < D / 2; d += 32) {
+          float acc = 0.f;
+#pragma unroll
+          for (int w = 0; w < kKeyWarps; ++w) acc += ow[(w * 8 + hh) * kLd + d] * f[w];
+          part[(prow + hh) * (D + 2) + 2 + hf * (D / 2) + d] = has ? acc : 0.f;
+        }
+      }
+      __syncthreads();
+    }
+    // The CTA that completes the row (the last of its CTAs to arrive) merges
+    // their partials into the output: O = sum_c o_c 2^(m_c - M) / sum_c l_c
+    // 2^(m_c - M), M the largest m_c.
+    __threadfence();
+    __syncthreads();
+    const long long r = static_cast<long long>(n) * Hkv + kvh;
+    if (tid == 0) {
+      const int nbl = __ldg(rowstart + n + 1) - __ldg(rowstart + n);
+      const long long s0 = static_cast<long long>(Hkv) * __ldg(rowstart + n) + static_cast<long long>(kvh) * nbl;
+      const int clo = share_owner(s0, T, P), chi = share_owner(s0 + nbl - 1, T, P);
+      // with T >= P every share holds a block; otherwise a share holds at most one
+      const unsigned expect = T >= P ? static_cast<unsigned>(chi - clo + 1) : static_cast<unsigned>(nbl);
+      ctl.clo = clo;
+      ctl.chi = chi;
+      ctl.last = atomicAdd(row_arrive + r, 1u) == expect - 1u;
+    }
+    __syncthreads();
+    if (ctl.last && hh < g) {
+      __threadfence();
+      const int clo = ctl.clo, chi = ctl.chi;
+      const float* pr = part + (r * g + hh) * (D + 2);   // + c g (D + 2) for CTA c
+      const long long cs_stride = static_cast<long long>(g) * (D + 2);
+      float Mx = -INFINITY;
+      for (int cc = clo + lane; cc <= chi; cc += 32)
+        if (share_start(cc, T, P) != share_start(cc + 1, T, P)) Mx = fmaxf(Mx, __ldcg(pr + cc * cs_stride));
+#pragma unroll
+      for (int x = 16; x > 0; x >>= 1) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, x));
+      float L = 0.f, O[D / 32];
+#pragma unroll
+      for (int k = 0; k < D / 32; ++k) O[k] = 0.f;
+      if (Mx > -INFINITY) {
+        for (int c0 = clo; c0 <= chi; c0 += 4) {   // four CTAs' partials in flight at once
+          float mk[4], lk[4], ok4[4][D / 32];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int cc = c0 + u;
+            const bool use = cc <= chi && share_start(cc, T, P) != share_start(cc + 1, T, P);
+            const float* pc = pr + (use ? cc : clo) * cs_stride;
+            mk[u] = use ? __ldcg(pc) : -INFINITY;
+            lk[u] = __ldcg(pc + 1);
+#pragma unroll
+            for (int k = 0; k < D / 32; ++k) ok4[u][k] = __ldcg(pc + 2 + lane + 32 * k);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float f = mk[u] > -INFINITY ? exp2f(mk[u] - Mx) : 0.f;
+            L += lk[u] * f;
+#pragma unroll
+            for (int k = 0; k < D / 32; ++k) O[k] += ok4[u][k] * f;
+          }
+        }
+      }
+      __nv_bfloat16* orow = o + (static_cast<long long>(n) * H + kvh * g + hh) * D;
+#pragma unroll
+      for (int k = 0; k < D / 32; ++k) orow[lane + 32 * k] = __float2bfloat16(L > 0.f ? O[k] / L : 0.f);
+    }
+    more = cs.next();
   }
-  __syncthreads();
-  // thread layout: head hh = tid / 32 (one warp per head), d columns lane, lane + 32, ...
-  const int hh = warp;
-  if (hh < g) {
-    const long long prow = ((static_cast<long long>(n) * H + kvh * g + hh) * NC + chunk) * (D + 2);
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kKeyWarps; ++w) M = fmaxf(M, ctl.ml[w][hh].x);
-    const bool has = done && M > -INFINITY;
-    float f[kKeyWarps], L = 0.f;
-#pragma unroll
-    for (int w = 0; w < kKeyWarps; ++w) {
-      const float2 ml = ctl.ml[w][hh];
-      f[w] = (has && ml.x > -INFINITY) ? exp2f(ml.x - M) : 0.f;
-      L += ml.y * f[w];
-    }
-    if (lane == 0) {
-      part[prow] = has ? M : -INFINITY;
-      part[prow + 1] = has ? L : 0.f;
-    }
-    for (int d = lane; d < D; d += 32) {
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kKeyWarps; ++w) acc += ow[(w * 8 + hh) * D + d] * f[w];
-      part[prow + 2 + d] = has ? acc : 0.f;
-    }
+  // copies still in flight land before the CTA exits (only after a wait ran out
+  // can any be left)
+  if (tid == 0) {
+    for (int i = max(seq, issued - kDecStages); i < issued; ++i)
+      drain_bar(smem_u32(&ctl.full[i % kDecStages]), (i / kDecStages) & 1, kDrainLimitNs);
   }
-}
-
-// Partials of the chunks of one (sequence, head) merged: O = sum_c o_c 2^(m_c - M)
-// / sum_c l_c 2^(m_c - M), M the largest m_c.  One thread per output column.
-template <int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ part, const int32_t* __restrict__ lens,
-                                                          int Lmax, int B, int NC, __nv_bfloat16* __restrict__ o) {
-  const int n = static_cast<int>(blockIdx.y);
-  const long long row = static_cast<long long>(n) * gridDim.x + blockIdx.x;   // n * H + h
-  const int c = threadIdx.x;
-  const int len = __ldg(lens + n);
-  const int nc = (len >= 1 && len <= Lmax) ? ((len - 1) / B) / kDecChunk + 1 : 0;
-  const float* p = part + row * NC * (D + 2);
-  float M = -INFINITY;
-  for (int k = 0; k < nc; ++k) M = fmaxf(M, p[k * (D + 2)]);
-  float L = 0.f, O = 0.f;
-  if (M > -INFINITY) {
-    for (int k = 0; k < nc; ++k) {
-      const float mk = p[k * (D + 2)];
-      if (mk == -INFINITY) continue;
-      const float f = exp2f(mk - M);
-      L += p[k * (D + 2) + 1] * f;
-      O += p[k * (D + 2) + 2 + c] * f;
-    }
-  }
-  o[row * D + c] = __float2bfloat16(L > 0.f ? O / L : 0.f);
 }
 
 template <int BN, int D>
@@ -664,6 +897,10 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
                             const DecodeScratch& w, const DeviceGuardArgs& g, cudaStream_t stream) {
   const int Nbm = Lmax / BN, W = (Nbm + 31) / 32;
   const float sl2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   CUtensorMap mks, mk, mv;
   const uint64_t rows = static_cast<uint64_t>(N) * Lmax;
   if (!make_tmap_sampled(&mks, k, rows, Hkv, D, S, kSearchTile) || !make_tmap_rows(&mk, k, rows, Hkv, D, BN) ||
@@ -671,11 +908,27 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
     return cudaErrorInvalidValue;
   constexpr int kSearchSmem = kSearchStages * kSearchTile * D * 2 + 1024;
   static std::atomic<uint64_t> search_smem_set{0};
-  cudaError_t e = set_smem_limit_once(decode_search_kernel<D>, kSearchSmem, search_smem_set);
-  if (e != cudaSuccess) return e;
-  decode_search_kernel<D><<<static_cast<unsigned>(N) * H, kDecThreads, kSearchSmem, stream>>>(
-      mks, static_cast<const __nv_bfloat16*>(q), lens, Lmax, H, Hkv, BN, S, sl2, tau, w.scores, Lmax / S, count, idx,
-      w.bits, Nbm, W, gqa ? w.mass : nullptr, g.status, g.limit_ns);
+  if ((e = set_smem_limit_once(decode_search_kernel<D>, kSearchSmem, search_smem_set)) != cudaSuccess) return e;
+  static std::atomic<int> search_occ{0};   // resident search CTAs per SM
+  int occ = search_occ.load(std::memory_order_relaxed);
+  if (occ == 0) {
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_search_kernel<D>, kDecThreads, kSearchSmem)) !=
+        cudaSuccess)
+      return e;
+    occ = std::max(occ, 1);
+    search_occ.store(occ, std::memory_order_relaxed);
+  }
+  // search: as many CTAs per row as keep the whole grid resident at once
+  const int Ns_max = Lmax / S, nt_max = (Ns_max + kSearchTile - 1) / kSearchTile;
+  const long long NH = static_cast<long long>(N) * H;
+  int SC = static_cast<int>(std::min<long long>(static_cast<long long>(occ) * sms / NH, kDecSearchChunks));
+  SC = std::max(1, std::min(SC, nt_max));
+  const int tpc = (nt_max + SC - 1) / SC;
+  SC = (nt_max + tpc - 1) / tpc;
+  decode_search_kernel<D><<<dim3(SC, static_cast<unsigned>(NH)), kDecThreads, kSearchSmem, stream>>>(
+      mks, static_cast<const __nv_bfloat16*>(q), lens, N, Lmax, H, Hkv, BN, S, sl2, tau, tpc, w.scores, Ns_max, w.cmax,
+      w.arrive, w.mass, gqa ? 1 : 0, count, idx, w.bits, Nbm, W, w.rowstart, static_cast<__nv_bfloat16*>(o),
+      g.status, g.limit_ns);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (gqa) {
     decode_group_select_kernel<<<static_cast<unsigned>(N) * Hkv, kDecThreads, 0, stream>>>(
@@ -685,12 +938,10 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
   using C = DecAttnCfg<BN, D>;
   static std::atomic<uint64_t> smem_set{0};
   if ((e = set_smem_limit_once(decode_attn_kernel<BN, D>, C::kSmem, smem_set)) != cudaSuccess) return e;
-  const int NC = (Nbm + kDecChunk - 1) / kDecChunk;
-  decode_attn_kernel<BN, D><<<dim3(NC, Hkv, N), kDecThreads, C::kSmem, stream>>>(
-      mk, mv, static_cast<const __nv_bfloat16*>(q), lens, w.bits, Lmax, H, Hkv, W, NC, sl2, w.part, g.status,
-      g.limit_ns);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  decode_combine_kernel<D><<<dim3(H, N), D, 0, stream>>>(w.part, lens, Lmax, BN, NC, static_cast<__nv_bfloat16*>(o));
+  const int P = std::max(1, std::min(sms, kDecAttnCTAs));
+  decode_attn_kernel<BN, D><<<P, kDecThreads, C::kSmem, stream>>>(
+      mk, mv, static_cast<const __nv_bfloat16*>(q), lens, w.rowstart, w.bits, N, Lmax, H, Hkv, W, sl2, w.part,
+      w.row_arrive, static_cast<__nv_bfloat16*>(o), g.status, g.limit_ns);
   return cudaGetLastError();
 }
 

@@ -132,24 +132,33 @@ HostLayout carve_host(int L, int H, int Hkv, int d, int B, int S) {
   return w;
 }
 
-// Decode workspace: the status word, the sampled scores [N, H, Lmax/S] fp32, the
-// kept-block bitmaps [N, H, W] u32 (W = ceil(Lmax/B / 32)) and the attention
-// partials [N, H, NC, d+2] fp32, one per 16-block chunk (NC = ceil(Lmax/B / 16)).
+// Decode workspace: the status word and the arrival counters of the search
+// (per sequence and head) and of the attention (per sequence and kv head), all
+// zeroed by one memset per call, the sampled scores [N, H, Lmax/S] fp32,
+// the kept-block bitmaps [N, H, W] u32 (W = ceil(Lmax/B / 32)), the attention
+// partials [(N Hkv + P) H/Hkv, d+2] fp32 (one per (row, attention CTA) pair, P
+// <= kDecAttnCTAs), the block masses [N, H, Lmax/B] fp32, the search CTAs' maxima
+// [N, H, kDecSearchChunks] fp32 and the prefix of block counts [N+1] i32.
 struct DecodeLayout {
-  size_t status, scores, bits, part, mass, total;
+  size_t status, arrive, row_arrive, zero_bytes, scores, bits, part, mass, cmax, rowstart, total;
 };
 
-DecodeLayout carve_decode(int N, int Lmax, int H, int d, int B, int S) {
+DecodeLayout carve_decode(int N, int Lmax, int H, int Hkv, int d, int B, int S) {
   DecodeLayout w;
   const size_t rows = static_cast<size_t>(N) * H;
   const size_t W = (static_cast<size_t>(Lmax / B) + 31) / 32;
-  const size_t NC = (static_cast<size_t>(Lmax / B) + 15) / 16;
-  size_t off = kAlign;
   w.status = 0;
+  w.arrive = 16;
+  w.row_arrive = w.arrive + rows * 4;
+  w.zero_bytes = w.row_arrive + static_cast<size_t>(N) * Hkv * 4;
+  size_t off = round_up(w.zero_bytes);
   w.scores = off; off += round_up(rows * (Lmax / S) * 4);
   w.bits = off; off += round_up(rows * W * 4);
-  w.part = off; off += round_up(rows * NC * (d + 2) * 4);
+  w.part = off;
+  off += round_up((static_cast<size_t>(N) * Hkv + rr::kDecAttnCTAs) * static_cast<size_t>(H / Hkv) * (d + 2) * 4);
   w.mass = off; off += round_up(rows * static_cast<size_t>(Lmax / B) * 4);
+  w.cmax = off; off += round_up(rows * rr::kDecSearchChunks * 4);
+  w.rowstart = off; off += round_up((static_cast<size_t>(N) + 1) * 4);
   w.total = off;
   return w;
 }
@@ -374,7 +383,7 @@ rr_status rr_decode_workspace_size(int N, int Lmax, int H, int Hkv, int d, int B
   if (!bytes) return RR_EINVAL;
   const rr_status st = check_decode_shape(N, Lmax, H, Hkv, d, B, S);
   if (st != RR_OK) return st;
-  *bytes = carve_decode(N, Lmax, H, d, B, S).total;
+  *bytes = carve_decode(N, Lmax, H, Hkv, d, B, S).total;
   return RR_OK;
 }
 
@@ -390,16 +399,19 @@ rr_status rr_decode_variant(const void* q, const void* k_cache, const void* v_ca
       !aligned16(idx) || (reinterpret_cast<uintptr_t>(lens) & 3u))
     return RR_EALIGN;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return RR_EALIGN;
-  const DecodeLayout w = carve_decode(N, Lmax, H, d, B, S);
+  const DecodeLayout w = carve_decode(N, Lmax, H, Hkv, d, B, S);
   if (workspace_bytes < w.total) return RR_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   unsigned int* status = reinterpret_cast<unsigned int*>(ws + w.status);
   const rr::DeviceGuardArgs g{status, g_wait_limit_ns};
-  const rr::DecodeScratch sc{reinterpret_cast<float*>(ws + w.scores), reinterpret_cast<uint32_t*>(ws + w.bits),
-                             reinterpret_cast<float*>(ws + w.part), reinterpret_cast<float*>(ws + w.mass)};
+  const rr::DecodeScratch sc{reinterpret_cast<float*>(ws + w.scores),       reinterpret_cast<uint32_t*>(ws + w.bits),
+                             reinterpret_cast<float*>(ws + w.part),         reinterpret_cast<float*>(ws + w.mass),
+                             reinterpret_cast<float*>(ws + w.cmax),         reinterpret_cast<unsigned int*>(ws + w.arrive),
+                             reinterpret_cast<unsigned int*>(ws + w.row_arrive),
+                             reinterpret_cast<int32_t*>(ws + w.rowstart)};
   const Range range("rr_decode");
-  if (cudaMemsetAsync(status, 0, sizeof(unsigned int), s) != cudaSuccess) return RR_ECUDA;
+  if (cudaMemsetAsync(ws, 0, w.zero_bytes, s) != cudaSuccess) return RR_ECUDA;   // status and arrival counters
   if (rr::launch_decode(q, k_cache, v_cache, lens, N, Lmax, H, Hkv, d, B, S, tau, (flags & RR_VAR_GQA_MASK) != 0,
                         count, idx, o, sc, g, s) != cudaSuccess)
     return RR_ECUDA;

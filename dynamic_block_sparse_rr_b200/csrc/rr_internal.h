@@ -95,11 +95,19 @@ constexpr unsigned kStatusLenCode = 8u;
 // partials [N, H, NC, d + 2] fp32 (max, sum, output columns per 16-block chunk,
 // NC = ceil(Lmax/B / 16)).
 struct DecodeScratch {
-  float* scores;
-  uint32_t* bits;
-  float* part;
-  float* mass;   // per-head block masses [N, H, Lmax/B] fp32 (one mask per GQA group only)
+  float* scores;          // sampled scores [N, H, Lmax/S] fp32
+  uint32_t* bits;         // kept-block bitmaps [N, H, W] u32
+  float* part;            // attention partials [(N Hkv + P) H/Hkv, d + 2] fp32
+  float* mass;            // block masses [N, H, Lmax/B] fp32
+  float* cmax;            // per search CTA: its max [N, H, kDecSearchChunks] fp32
+  unsigned int* arrive;   // per (sequence, head): search CTAs done [N, H] u32, zero before the launch
+  unsigned int* row_arrive;   // per (sequence, kv head): attention CTAs done [N, Hkv] u32, zero before the launch
+  int32_t* rowstart;      // prefix of the sequences' block counts [N + 1] i32
 };
+
+// Search CTAs per (sequence, head) and attention CTAs per launch, at most.
+constexpr int kDecSearchChunks = 32;
+constexpr int kDecAttnCTAs = 1024;
 
 // Decode stage: search, block-sparse attention and combine for one new token per
 // sequence.  q, o: [N, H, d]; k, v: [N, Lmax, Hkv, d]; lens: [N] cache lengths.

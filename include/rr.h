@@ -202,16 +202,18 @@ rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int 
  *      lens[n]-1; lens [N] int32 (device), each in [1, Lmax].
  * Out: count [N,H] int32, idx [N,H,Lmax/B] int32 (kept blocks ascending, valid
  *      below count), o [N,H,d] bf16.  All device memory, caller-owned.
- * Workspace: rr_decode_workspace_size bytes, 256-byte aligned (sampled scores,
- * kept-block bitmaps, per-chunk attention partials, per-head block masses,
- * status word).
+ * Workspace: rr_decode_workspace_size bytes, 256-byte aligned (status word
+ * and arrival counters, zeroed by the call; sampled scores, kept-block
+ * bitmaps, attention partials, block masses, the prefix of the sequences'
+ * block counts).  One call at a time per workspace.
  * Requires Lmax % B == 0, B % S == 0, d and B in {64, 128}, H/Hkv <= 8,
  * Lmax/B <= 4096.  A length outside [1, Lmax] is found on the device: that
  * sequence gets count 0 and a zero output, and rr_check_status returns
- * RR_EINVAL.  Kernels: a search CTA per (sequence, head), an attention CTA per
- * (sequence, kv head, 16 key blocks) that loads each kept K/V block once for
- * every head of its GQA group that kept it, and a combine CTA per
- * (sequence, head). */
+ * RR_EINVAL.  Kernels: search CTAs over runs of each (sequence, head)'s
+ * sampled keys, the last of a row's CTAs selecting; then one attention CTA
+ * per SM over an equal share of all causal key blocks of all sequences and kv
+ * heads, which loads each kept K/V block once for every head of its GQA group
+ * that kept it, the last CTA of a (sequence, kv head) merging the partials. */
 rr_status rr_decode_workspace_size(int N, int Lmax, int H, int Hkv, int d, int B, int S, size_t* bytes);
 rr_status rr_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int N, int Lmax,
                     int H, int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,

@@ -125,6 +125,22 @@ def test_decode_gqa_group_mask(rr, structure, H, Hkv, tau):
              flags=rr.VAR_GQA_MASK)
 
 
+def test_decode_many_ragged_sequences(rr):
+    """Thirty-seven sequences of very different lengths (one key, one block, a
+    block and one key, full caches, the rest seeded): the attention CTAs' shares
+    of the flattened (sequence, kv head, block) space cut rows at arbitrary
+    blocks and span several short rows each."""
+    rng = np.random.default_rng(23)
+    lens = [1, 128, 129, 2048, 2047, 5] + [int(x) for x in rng.integers(1, 2049, 31)]
+    run_case(rr, len(lens), 2048, 8, 2, 128, 128, 16, 0.9, lens, seed=29)
+
+
+def test_decode_single_short_sequence(rr):
+    """One sequence inside its first block: fewer flattened blocks than attention
+    CTAs, so most CTAs have an empty share."""
+    run_case(rr, 1, 1024, 4, 1, 128, 128, 16, 0.9, [100], seed=31)
+
+
 def test_decode_tau_one_is_dense(rr):
     lens = [3000, 4096, 17]
     count, idx = run_case(rr, 3, 4096, 4, 2, 128, 128, 16, 1.0, lens, seed=7)
