@@ -271,7 +271,7 @@ __device__ void block_count_prefix(const int32_t* __restrict__ lens, int N, int 
   if (threadIdx.x == 0) rowstart[N] = static_cast<int32_t>(carry);
 }
 
-// grid (SC, N*H): CTA (c, row) scores the sampled keys of tiles [c tpc, (c+1) tpc)
+// grid (N*H, SC): CTA (row, c) scores the sampled keys of tiles [c tpc, (c+1) tpc)
 // of its (sequence, head) row and owns the key blocks those keys fall in
 // (B/S divides the 128 strides of a tile).  Its max and its blocks' masses on
 // that max go to the workspace; the CTA that arrives last on the row's counter
@@ -290,8 +290,8 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_search_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
-  const int SC = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-  const long long row = blockIdx.y;
+  const int SC = static_cast<int>(gridDim.y), c = static_cast<int>(blockIdx.y);
+  const long long row = blockIdx.x;
   const int n = static_cast<int>(row / H), h = static_cast<int>(row % H);
   const int kvh = h / (H / Hkv);
   int32_t* out = idx + row * Nbm;
@@ -925,7 +925,7 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
   SC = std::max(1, std::min(SC, nt_max));
   const int tpc = (nt_max + SC - 1) / SC;
   SC = (nt_max + tpc - 1) / tpc;
-  decode_search_kernel<D><<<dim3(SC, static_cast<unsigned>(NH)), kDecThreads, kSearchSmem, stream>>>(
+  decode_search_kernel<D><<<dim3(static_cast<unsigned>(NH), SC), kDecThreads, kSearchSmem, stream>>>(
       mks, static_cast<const __nv_bfloat16*>(q), lens, N, Lmax, H, Hkv, BN, S, sl2, tau, tpc, w.scores, Ns_max, w.cmax,
       w.arrive, w.mass, gqa ? 1 : 0, count, idx, w.bits, Nbm, W, w.rowstart, static_cast<__nv_bfloat16*>(o),
       g.status, g.limit_ns);

@@ -44,7 +44,7 @@ def _make(N, Lmax, H, Hkv, d, structure, seed):
     return qs, np.stack(ks), np.stack(vs)
 
 
-def run_case(rr, N, Lmax, H, Hkv, d, B, S, tau, lens, structure=gen.PLANTED, seed=0, flags=0):
+def run_case(rr, N, Lmax, H, Hkv, d, B, S, tau, lens, structure=gen.PLANTED, seed=0, flags=0, check=None):
     Qs, K, V = _make(N, Lmax, H, Hkv, d, structure, seed)
     q = np.stack([Qs[n][lens[n] - 1] for n in range(N)])              # [N, H, d]
     qd, kd, vd = _bf16(q).cuda(), _bf16(K).cuda(), _bf16(V).cuda()
@@ -56,7 +56,7 @@ def run_case(rr, N, Lmax, H, Hkv, d, B, S, tau, lens, structure=gen.PLANTED, see
     count, idx, og = count.cpu().numpy(), idx.cpu().numpy(), o.float().cpu().numpy()
     stats = {"rows_differing": 0, "band": 0, "tie": 0, "fail": 0}
     errs = []
-    for n in range(N):
+    for n in (range(N) if check is None else check):
         t = lens[n] - 1
         Jt = t // B
         M = oracle.decode_block_mass(q[n], K[n], t, B, S)
@@ -89,6 +89,7 @@ def run_case(rr, N, Lmax, H, Hkv, d, B, S, tau, lens, structure=gen.PLANTED, see
     assert stats["fail"] == 0, stats
     err = np.concatenate([e.ravel() for e in errs])
     assert err.max() <= MAX_ERR and err.mean() <= MEAN_ERR, (err.max(), err.mean())
+    assert np.all(count >= 1) and np.all(np.isfinite(og))
     visited = float(count.sum()) / sum(H * ((l - 1) // B + 1) for l in lens)
     print({"stats": stats, "max_err": float(err.max()), "mean_err": float(err.mean()), "visited": visited})
     return count, idx
@@ -139,6 +140,46 @@ def test_decode_single_short_sequence(rr):
     """One sequence inside its first block: fewer flattened blocks than attention
     CTAs, so most CTAs have an empty share."""
     run_case(rr, 1, 1024, 4, 1, 128, 128, 16, 0.9, [100], seed=31)
+
+
+def test_decode_more_rows_than_a_grid_dimension_holds(rr):
+    """4100 sequences x 16 heads = 65 600 (sequence, head) rows, more than the
+    65 535 of a grid's y or z dimension.  Caches of 256 keys (four 64-key
+    blocks), seeded lengths; a seeded sample of 40 sequences, the first and the
+    last among them, against the oracle, and every row checked for a non-empty
+    list ending at its current block and a finite output."""
+    N, Lmax, H, Hkv, d, B, S, tau = 4100, 256, 16, 2, 64, 64, 4, 0.9
+    rng = np.random.default_rng(37)
+    lens = [int(x) for x in rng.integers(1, Lmax + 1, N)]
+    # one query row per sequence, and the caches, straight from the generator
+    q = gen.bf16_bits_to_f32(gen.fill(gen.IID, 41, gen.ROLE_Q, N, H, Hkv, d))
+    K = gen.bf16_bits_to_f32(gen.fill(gen.IID, 41, gen.ROLE_K, N * Lmax, H, Hkv, d)).reshape(N, Lmax, Hkv, d)
+    V = gen.bf16_bits_to_f32(gen.fill(gen.IID, 41, gen.ROLE_V, N * Lmax, H, Hkv, d)).reshape(N, Lmax, Hkv, d)
+    ws = torch.empty(rr.decode_workspace_size(N, Lmax, H, Hkv, d, B, S), dtype=torch.uint8, device="cuda")
+    o, count, idx = rr.decode(_bf16(q).cuda(), _bf16(K).cuda(), _bf16(V).cuda(),
+                              torch.tensor(lens, dtype=torch.int32, device="cuda"), B, S, tau, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+    count, idx, og = count.cpu().numpy(), idx.cpu().numpy(), o.float().cpu().numpy()
+    last = np.array([(l - 1) // B for l in lens])
+    assert np.all(count >= 1) and np.all(np.isfinite(og))
+    assert np.all(idx[np.arange(N)[:, None], np.arange(H)[None, :], count - 1] == last[:, None])
+    check = sorted({0, N - 1} | {int(x) for x in rng.choice(N, 38, replace=False)})
+    fails = 0
+    for n in check:
+        t = lens[n] - 1
+        M = oracle.decode_block_mass(q[n], K[n], t, B, S)
+        blocks = []
+        for h in range(H):
+            g_sel = idx[n, h, :count[n, h]]
+            o_sel = oracle.decode_select(M[h], t // B, tau)
+            diff = set(g_sel.tolist()) ^ set(o_sel.tolist())
+            if diff:
+                near, ties = oracle.decode_band_blocks(M[h], t // B, tau)
+                fails += len(diff - near - ties)
+            blocks.append(g_sel)
+        ref = oracle.decode_attention(q[n], K[n], V[n], t, blocks, B)
+        assert np.abs(og[n] - ref).max() <= MAX_ERR, n
+    assert fails == 0
 
 
 def test_decode_tau_one_is_dense(rr):
