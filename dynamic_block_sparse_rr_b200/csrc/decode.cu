@@ -26,7 +26,7 @@
 //   decode_attn_kernel     one persistent CTA per SM over an equal share of the
 //                          flattened (sequence, kv head, causal key block)
 //                          space: a kept block's K and V tiles come in once by
-//                          TMA (three-stage ring, running on across rows) for
+//                          TMA (two-stage ring, running on across rows) for
 //                          every query head of the GQA group that kept it.  The
 //                          group's <= 8 heads are the 8 columns of m16n8k16
 //                          tiles, so the two small contractions per block
@@ -34,8 +34,9 @@
 //                          warp; each warp keeps an online softmax over its 16
 //                          keys of every block.  At the end of each row the
 //                          warps' partials merge into the CTA's partial for the
-//                          row, and the last of the row's CTAs to finish merges
-//                          those into the output.
+//                          row;
+//   decode_combine_kernel  one CTA per (sequence, kv head): the partials of the
+//                          CTAs that shared the row merged into the output.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_search_kernel(
     int N, int Lmax, int H, int Hkv, int B, int S, float sl2, float tau, int tpc, float* __restrict__ scores,
     int Ns_max, float* __restrict__ cmax, unsigned int* __restrict__ arrive, float* __restrict__ mass, int group,
     int32_t* __restrict__ count, int32_t* __restrict__ idx, uint32_t* __restrict__ bits, int Nbm, int W,
-    int32_t* __restrict__ rowstart, __nv_bfloat16* __restrict__ o, unsigned int* status, uint64_t limit_ns) {
+    int32_t* __restrict__ rowstart, unsigned int* status, uint64_t limit_ns) {
   constexpr int kTileBytes = kSearchTile * D * 2;
   static_assert(kMaxBlocks * 4 + kMaxBlocks / 8 <= kSearchStages * kTileBytes, "selection arrays fit in the ring");
   __shared__ DecSearchShared sh;
@@ -298,9 +299,8 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_search_kernel(
   uint32_t* obits = bits + row * W;
   if (c == 0 && row == 0) block_count_prefix(lens, N, Lmax, B, rowstart, sh.ubuf);
   const int len = __ldg(lens + n);
-  if (len < 1 || len > Lmax) {   // not a cache length this call can serve: nothing selected, zero output
+  if (len < 1 || len > Lmax) {   // not a cache length this call can serve: nothing selected
     if (c == 0) {
-      for (int k = tid; k < D; k += kDecThreads) o[row * D + k] = __float2bfloat16(0.f);
       if (tid == 0) {
         count[row] = 0;
         atomicCAS(status, 0u, kStatusLenCode | (static_cast<unsigned>(n < (1 << 24) ? n : (1 << 24) - 1) << 8));
@@ -461,7 +461,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_select_kernel(const 
 }
 
 // ------------------------------------------------------------------ attention
-constexpr int kDecStages = 3;
+constexpr int kDecStages = 2;
 
 template <int BN, int D>
 struct DecAttnCfg {
@@ -475,8 +475,6 @@ struct DecAttnCfg {
 struct DecAttnCtrl {
   uint64_t full[kDecStages];
   int abort;
-  int last;                                // this CTA completes the current row
-  int clo, chi;                            // the CTAs whose shares meet the current row
   float2 ml[kDecWarps][8];                 // warp partials: (max, sum) per head
   __nv_bfloat16 p[kDecWarps][8][24];       // per warp: P of its 16 keys, [head][key] (rows padded)
 };
@@ -610,7 +608,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
     const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lens, const int32_t* __restrict__ rowstart,
     const uint32_t* __restrict__ bits, int N, int Lmax, int H, int Hkv, int W, float sl2, float* __restrict__ part,
-    unsigned int* __restrict__ row_arrive, __nv_bfloat16* __restrict__ o, unsigned int* status, uint64_t limit_ns) {
+    unsigned int* status, uint64_t limit_ns) {
   using C = DecAttnCfg<BN, D>;
   constexpr int kKeyWarps = BN / 16;  // warps that own keys (8 at B = 128, 4 at B = 64)
   constexpr int kDSteps = D / 16;     // k-steps of S (over d)
@@ -825,62 +823,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
       }
       __syncthreads();
     }
-    // The CTA that completes the row (the last of its CTAs to arrive) merges
-    // their partials into the output: O = sum_c o_c 2^(m_c - M) / sum_c l_c
-    // 2^(m_c - M), M the largest m_c.
-    __threadfence();
-    __syncthreads();
-    const long long r = static_cast<long long>(n) * Hkv + kvh;
-    if (tid == 0) {
-      const int nbl = __ldg(rowstart + n + 1) - __ldg(rowstart + n);
-      const long long s0 = static_cast<long long>(Hkv) * __ldg(rowstart + n) + static_cast<long long>(kvh) * nbl;
-      const int clo = share_owner(s0, T, P), chi = share_owner(s0 + nbl - 1, T, P);
-      // with T >= P every share holds a block; otherwise a share holds at most one
-      const unsigned expect = T >= P ? static_cast<unsigned>(chi - clo + 1) : static_cast<unsigned>(nbl);
-      ctl.clo = clo;
-      ctl.chi = chi;
-      ctl.last = atomicAdd(row_arrive + r, 1u) == expect - 1u;
-    }
-    __syncthreads();
-    if (ctl.last && hh < g) {
-      __threadfence();
-      const int clo = ctl.clo, chi = ctl.chi;
-      const float* pr = part + (r * g + hh) * (D + 2);   // + c g (D + 2) for CTA c
-      const long long cs_stride = static_cast<long long>(g) * (D + 2);
-      float Mx = -INFINITY;
-      for (int cc = clo + lane; cc <= chi; cc += 32)
-        if (share_start(cc, T, P) != share_start(cc + 1, T, P)) Mx = fmaxf(Mx, __ldcg(pr + cc * cs_stride));
-#pragma unroll
-      for (int x = 16; x > 0; x >>= 1) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, x));
-      float L = 0.f, O[D / 32];
-#pragma unroll
-      for (int k = 0; k < D / 32; ++k) O[k] = 0.f;
-      if (Mx > -INFINITY) {
-        for (int c0 = clo; c0 <= chi; c0 += 4) {   // four CTAs' partials in flight at once
-          float mk[4], lk[4], ok4[4][D / 32];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int cc = c0 + u;
-            const bool use = cc <= chi && share_start(cc, T, P) != share_start(cc + 1, T, P);
-            const float* pc = pr + (use ? cc : clo) * cs_stride;
-            mk[u] = use ? __ldcg(pc) : -INFINITY;
-            lk[u] = __ldcg(pc + 1);
-#pragma unroll
-            for (int k = 0; k < D / 32; ++k) ok4[u][k] = __ldcg(pc + 2 + lane + 32 * k);
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float f = mk[u] > -INFINITY ? exp2f(mk[u] - Mx) : 0.f;
-            L += lk[u] * f;
-#pragma unroll
-            for (int k = 0; k < D / 32; ++k) O[k] += ok4[u][k] * f;
-          }
-        }
-      }
-      __nv_bfloat16* orow = o + (static_cast<long long>(n) * H + kvh * g + hh) * D;
-#pragma unroll
-      for (int k = 0; k < D / 32; ++k) orow[lane + 32 * k] = __float2bfloat16(L > 0.f ? O[k] / L : 0.f);
-    }
     more = cs.next();
   }
   // copies still in flight land before the CTA exits (only after a wait ran out
@@ -888,6 +830,102 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
   if (tid == 0) {
     for (int i = max(seq, issued - kDecStages); i < issued; ++i)
       drain_bar(smem_u32(&ctl.full[i % kDecStages]), (i / kDecStages) & 1, kDrainLimitNs);
+  }
+}
+
+// The partials of the attention CTAs whose shares met row (n, kvh) merged into
+// the output of the group's g heads: O = sum_c o_c 2^(m_c - M) / sum_c l_c
+// 2^(m_c - M), M the largest m_c.  One CTA per row.  The row's g * D outputs are
+// split into runs of 4 adjacent columns over nthr = g * D / 4 threads; the
+// CTA's 256 threads form 256 / nthr groups (1 to 16) that merge disjoint runs
+// of the row's partials, each run's loads (up to 16 partials) in flight at
+// once; the groups' (max, sum, output) states combine through shared memory.
+// A sequence with no blocks (a length outside [1, Lmax]) gets a zero output.
+template <int D>
+__global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const float* __restrict__ part,
+                                                                    const int32_t* __restrict__ rowstart, int N,
+                                                                    int H, int Hkv, int P,
+                                                                    __nv_bfloat16* __restrict__ o) {
+  constexpr int kBatch = 16;
+  __shared__ float4 gs[2 * kDecThreads];   // per group and thread: (max, sum, o0, o1) and (o2, o3)
+  const int tid = threadIdx.x;
+  const long long r = blockIdx.x;
+  const int n = static_cast<int>(r / Hkv), kvh = static_cast<int>(r % Hkv);
+  const int g = H / Hkv;
+  const int nthr = g * D / 4, groups = kDecThreads / nthr;
+  const int grp = tid / nthr, e0 = 4 * (tid % nthr);
+  const int hm = e0 / D, col = e0 % D;
+  const int nbl = __ldg(rowstart + n + 1) - __ldg(rowstart + n);
+  float Mx = -INFINITY, L = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
+  if (nbl > 0) {
+    const long long T = static_cast<long long>(Hkv) * __ldg(rowstart + N);
+    const long long s0 = static_cast<long long>(Hkv) * __ldg(rowstart + n) + static_cast<long long>(kvh) * nbl;
+    const int clo = share_owner(s0, T, P), chi = share_owner(s0 + nbl - 1, T, P);
+    const int per = (chi - clo + 1 + groups - 1) / groups;
+    const int g0 = clo + grp * per, g1 = min(g0 + per, chi + 1);
+    const float* pr = part + (r * g + hm) * (D + 2);   // + c g (D + 2) for CTA c
+    const long long cs_stride = static_cast<long long>(g) * (D + 2);
+    // with T >= P every share holds a block (and the 64-bit divisions of the
+    // test stay out of the loop); otherwise an empty share wrote nothing
+    const bool all_full = T >= P;
+    for (int base = g0; base < g1; base += kBatch) {
+      float mk[kBatch], lk[kBatch];
+      float2 ok[kBatch][2];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int cc = base + u;
+        const bool use = cc < g1 && (all_full || share_start(cc, T, P) != share_start(cc + 1, T, P));
+        const float* pc = pr + static_cast<long long>(use ? cc : clo) * cs_stride;
+        mk[u] = __ldg(pc);
+        lk[u] = __ldg(pc + 1);
+        ok[u][0] = __ldg(reinterpret_cast<const float2*>(pc + 2 + col));
+        ok[u][1] = __ldg(reinterpret_cast<const float2*>(pc + 4 + col));
+        if (!use) mk[u] = -INFINITY;
+      }
+      float bm = Mx;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) bm = fmaxf(bm, mk[u]);
+      if (bm == -INFINITY) continue;
+      const float a = Mx == -INFINITY ? 0.f : exp2f(Mx - bm);
+      L *= a;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) O[k] *= a;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const float f = mk[u] == -INFINITY ? 0.f : exp2f(mk[u] - bm);
+        L += lk[u] * f;
+        O[0] += ok[u][0].x * f;
+        O[1] += ok[u][0].y * f;
+        O[2] += ok[u][1].x * f;
+        O[3] += ok[u][1].y * f;
+      }
+      Mx = bm;
+    }
+  }
+  if (grp < groups) {
+    gs[grp * nthr + tid % nthr] = make_float4(Mx, L, O[0], O[1]);
+    gs[kDecThreads + grp * nthr + tid % nthr] = make_float4(O[2], O[3], 0.f, 0.f);
+  }
+  __syncthreads();
+  if (tid < nthr) {
+    float M = -INFINITY;
+    for (int k = 0; k < groups; ++k) M = fmaxf(M, gs[k * nthr + tid].x);
+    float Ls = 0.f, A[4] = {0.f, 0.f, 0.f, 0.f};
+    if (M > -INFINITY) {
+      for (int k = 0; k < groups; ++k) {
+        const float4 st = gs[k * nthr + tid], s2 = gs[kDecThreads + k * nthr + tid];
+        const float f = st.x == -INFINITY ? 0.f : exp2f(st.x - M);
+        Ls += st.y * f;
+        A[0] += st.z * f;
+        A[1] += st.w * f;
+        A[2] += s2.x * f;
+        A[3] += s2.y * f;
+      }
+    }
+    const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
+    __nv_bfloat16* orow = o + (static_cast<long long>(n) * H + kvh * g + hm) * D + col;
+    *reinterpret_cast<__nv_bfloat162*>(orow) = __floats2bfloat162_rn(A[0] * inv, A[1] * inv);
+    *reinterpret_cast<__nv_bfloat162*>(orow + 2) = __floats2bfloat162_rn(A[2] * inv, A[3] * inv);
   }
 }
 
@@ -927,8 +965,7 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
   SC = (nt_max + tpc - 1) / tpc;
   decode_search_kernel<D><<<dim3(static_cast<unsigned>(NH), SC), kDecThreads, kSearchSmem, stream>>>(
       mks, static_cast<const __nv_bfloat16*>(q), lens, N, Lmax, H, Hkv, BN, S, sl2, tau, tpc, w.scores, Ns_max, w.cmax,
-      w.arrive, w.mass, gqa ? 1 : 0, count, idx, w.bits, Nbm, W, w.rowstart, static_cast<__nv_bfloat16*>(o),
-      g.status, g.limit_ns);
+      w.arrive, w.mass, gqa ? 1 : 0, count, idx, w.bits, Nbm, W, w.rowstart, g.status, g.limit_ns);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (gqa) {
     decode_group_select_kernel<<<static_cast<unsigned>(N) * Hkv, kDecThreads, 0, stream>>>(
@@ -941,7 +978,10 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
   const int P = std::max(1, std::min(sms, kDecAttnCTAs));
   decode_attn_kernel<BN, D><<<P, kDecThreads, C::kSmem, stream>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(q), lens, w.rowstart, w.bits, N, Lmax, H, Hkv, W, sl2, w.part,
-      w.row_arrive, static_cast<__nv_bfloat16*>(o), g.status, g.limit_ns);
+      g.status, g.limit_ns);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  decode_combine_kernel<D><<<static_cast<unsigned>(N) * Hkv, kDecThreads, 0, stream>>>(
+      w.part, w.rowstart, N, H, Hkv, P, static_cast<__nv_bfloat16*>(o));
   return cudaGetLastError();
 }
 

@@ -132,15 +132,14 @@ HostLayout carve_host(int L, int H, int Hkv, int d, int B, int S) {
   return w;
 }
 
-// Decode workspace: the status word and the arrival counters of the search
-// (per sequence and head) and of the attention (per sequence and kv head), all
-// zeroed by one memset per call, the sampled scores [N, H, Lmax/S] fp32,
+// Decode workspace: the status word and the search's arrival counters (per
+// sequence and head), zeroed by one memset per call, the sampled scores [N, H, Lmax/S] fp32,
 // the kept-block bitmaps [N, H, W] u32 (W = ceil(Lmax/B / 32)), the attention
 // partials [(N Hkv + P) H/Hkv, d+2] fp32 (one per (row, attention CTA) pair, P
 // <= kDecAttnCTAs), the block masses [N, H, Lmax/B] fp32, the search CTAs' maxima
 // [N, H, kDecSearchChunks] fp32 and the prefix of block counts [N+1] i32.
 struct DecodeLayout {
-  size_t status, arrive, row_arrive, zero_bytes, scores, bits, part, mass, cmax, rowstart, total;
+  size_t status, arrive, zero_bytes, scores, bits, part, mass, cmax, rowstart, total;
 };
 
 DecodeLayout carve_decode(int N, int Lmax, int H, int Hkv, int d, int B, int S) {
@@ -149,8 +148,7 @@ DecodeLayout carve_decode(int N, int Lmax, int H, int Hkv, int d, int B, int S) 
   const size_t W = (static_cast<size_t>(Lmax / B) + 31) / 32;
   w.status = 0;
   w.arrive = 16;
-  w.row_arrive = w.arrive + rows * 4;
-  w.zero_bytes = w.row_arrive + static_cast<size_t>(N) * Hkv * 4;
+  w.zero_bytes = w.arrive + rows * 4;
   size_t off = round_up(w.zero_bytes);
   w.scores = off; off += round_up(rows * (Lmax / S) * 4);
   w.bits = off; off += round_up(rows * W * 4);
@@ -408,7 +406,6 @@ rr_status rr_decode_variant(const void* q, const void* k_cache, const void* v_ca
   const rr::DecodeScratch sc{reinterpret_cast<float*>(ws + w.scores),       reinterpret_cast<uint32_t*>(ws + w.bits),
                              reinterpret_cast<float*>(ws + w.part),         reinterpret_cast<float*>(ws + w.mass),
                              reinterpret_cast<float*>(ws + w.cmax),         reinterpret_cast<unsigned int*>(ws + w.arrive),
-                             reinterpret_cast<unsigned int*>(ws + w.row_arrive),
                              reinterpret_cast<int32_t*>(ws + w.rowstart)};
   const Range range("rr_decode");
   if (cudaMemsetAsync(ws, 0, w.zero_bytes, s) != cudaSuccess) return RR_ECUDA;   // status and arrival counters

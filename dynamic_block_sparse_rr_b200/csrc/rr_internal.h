@@ -101,7 +101,6 @@ struct DecodeScratch {
   float* mass;            // block masses [N, H, Lmax/B] fp32
   float* cmax;            // per search CTA: its max [N, H, kDecSearchChunks] fp32
   unsigned int* arrive;   // per (sequence, head): search CTAs done [N, H] u32, zero before the launch
-  unsigned int* row_arrive;   // per (sequence, kv head): attention CTAs done [N, Hkv] u32, zero before the launch
   int32_t* rowstart;      // prefix of the sequences' block counts [N + 1] i32
 };
 

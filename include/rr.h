@@ -213,7 +213,7 @@ rr_status rr_mask_to_dense(const int32_t* count, const int32_t* idx, int H, int 
  * sampled keys, the last of a row's CTAs selecting; then one attention CTA
  * per SM over an equal share of all causal key blocks of all sequences and kv
  * heads, which loads each kept K/V block once for every head of its GQA group
- * that kept it, the last CTA of a (sequence, kv head) merging the partials. */
+ * that kept it; then one CTA per (sequence, kv head) merging the partials. */
 rr_status rr_decode_workspace_size(int N, int Lmax, int H, int Hkv, int d, int B, int S, size_t* bytes);
 rr_status rr_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int N, int Lmax,
                     int H, int Hkv, int d, int B, int S, float tau, int32_t* count, int32_t* idx, void* o,
