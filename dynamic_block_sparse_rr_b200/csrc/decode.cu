@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_search_kernel(
     int32_t* __restrict__ count, int32_t* __restrict__ idx, uint32_t* __restrict__ bits, int Nbm, int W,
     int32_t* __restrict__ rowstart, unsigned int* status, uint64_t limit_ns) {
   constexpr int kTileBytes = kSearchTile * D * 2;
-  static_assert(kMaxBlocks * 4 + kMaxBlocks / 8 <= kSearchStages * kTileBytes, "selection arrays fit in the ring");
+  static_assert(kMaxBlocks * 4 + kMaxBlocks / 8 + kDecSearchChunks * 4 <= kSearchStages * kTileBytes,
+                "selection arrays fit in the ring");
   __shared__ DecSearchShared sh;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -409,11 +410,26 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_search_kernel(
   // shared memory (every copy has landed)
   float* smass = reinterpret_cast<float*>(smem);
   uint32_t* swbits = reinterpret_cast<uint32_t*>(smem + kMaxBlocks * 4);
+  float* scm = reinterpret_cast<float*>(smem + kMaxBlocks * 4 + kMaxBlocks / 8);
+  // one round of loads (a load here waits behind the other CTAs' stream): the
+  // runs' maxima and this thread's masses
+  if (tid < SC) scm[tid] = __ldcg(cmax + row * SC + tid);
+  float mv[kMaxPer];
+#pragma unroll
+  for (int e = 0; e < kMaxPer; ++e) {
+    const int J = tid + e * kDecThreads;
+    mv[e] = J < nb ? __ldcg(mrow + J) : 0.f;
+  }
+  __syncthreads();
   float M = -INFINITY;
-  for (int k = 0; k < SC; ++k) M = fmaxf(M, __ldcg(cmax + row * SC + k));
-  for (int J = tid; J < nb; J += kDecThreads) {
-    const float ck = __ldcg(cmax + row * SC + J / bpc);
-    smass[J] = ck > -INFINITY ? __ldcg(mrow + J) * exp2f(ck - M) : 0.f;
+  for (int k = 0; k < SC; ++k) M = fmaxf(M, scm[k]);
+#pragma unroll
+  for (int e = 0; e < kMaxPer; ++e) {
+    const int J = tid + e * kDecThreads;
+    if (J < nb) {
+      const float ck = scm[J / bpc];
+      smass[J] = ck > -INFINITY ? mv[e] * exp2f(ck - M) : 0.f;
+    }
   }
   __syncthreads();
 
