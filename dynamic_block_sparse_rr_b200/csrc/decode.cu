@@ -384,6 +384,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_search_kernel(
     for (int i = (issued - i0 > kSearchStages ? issued - kSearchStages : i0); i < issued; ++i)
       drain_bar(smem_u32(&sh.full[(i - i0) % kSearchStages]), ((i - i0) / kSearchStages) & 1, kDrainLimitNs);
   }
+  grid_dependents_launch();   // the next grid may take the SMs this one frees
   // a wait that ran out (status recorded) leaves this run without mass
   const bool good = __syncthreads_and(ok);
   const float cm = good ? block_max(lmax, sh.fbuf) : -INFINITY;
@@ -506,8 +507,8 @@ struct SegWalk {
   long long pos, b1;
   int n, kvh, Ja, Jb;
   __device__ __forceinline__ void load() {
-    const long long base = static_cast<long long>(Hkv) * __ldg(rs + n);
-    const int nbl = __ldg(rs + n + 1) - __ldg(rs + n);
+    const long long base = static_cast<long long>(Hkv) * __ldcg(rs + n);
+    const int nbl = __ldcg(rs + n + 1) - __ldcg(rs + n);
     const long long o = pos - base;
     kvh = static_cast<int>(o / nbl);
     Ja = static_cast<int>(o % nbl);
@@ -524,7 +525,7 @@ struct SegWalk {
     int lo = 0, hi = N - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (static_cast<long long>(Hkv) * __ldg(rs + mid) <= pos) lo = mid;
+      if (static_cast<long long>(Hkv) * __ldcg(rs + mid) <= pos) lo = mid;
       else hi = mid - 1;
     }
     n = lo;
@@ -534,9 +535,9 @@ struct SegWalk {
   __device__ bool next() {
     pos += Jb - Ja;
     if (pos >= b1) return false;
-    if (pos == static_cast<long long>(Hkv) * __ldg(rs + n + 1)) {   // the next sequence with blocks
+    if (pos == static_cast<long long>(Hkv) * __ldcg(rs + n + 1)) {   // the next sequence with blocks
       do ++n;
-      while (__ldg(rs + n + 1) == __ldg(rs + n));
+      while (__ldcg(rs + n + 1) == __ldcg(rs + n));
     }
     load();
     return true;
@@ -553,7 +554,7 @@ __device__ __forceinline__ uint32_t group_word(const uint32_t* __restrict__ bits
                                                int W, int w) {
   const uint32_t* b = bits + (static_cast<long long>(s.n) * H + s.kvh * g) * W + w;
   uint32_t u = 0u;
-  for (int hh = 0; hh < g; ++hh) u |= __ldg(b + static_cast<long long>(hh) * W);
+  for (int hh = 0; hh < g; ++hh) u |= __ldcg(b + static_cast<long long>(hh) * W);
   return u & seg_mask(s, w);
 }
 
@@ -639,14 +640,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
   const int gid = lane >> 2, tig = lane & 3;   // mma fragment coordinates
   const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   const int g = H / Hkv;
-  const long long T = static_cast<long long>(Hkv) * __ldg(rowstart + N);
-  const long long b0 = share_start(c, T, P), b1 = share_start(c + 1, T, P);
-  if (b0 >= b1) return;
   if (tid == 0) {
     for (int st = 0; st < kDecStages; ++st) mbar_init(smem_u32(&ctl.full[st]), 1);
     ctl.abort = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&mk);
+    tma_prefetch_desc(&mv);
   }
+  // the search's lists and block-count prefix (the grid ahead, launched so that
+  // this one may start early) are read only past this point, through L2
+  grid_dependency_wait();
+  const long long T = static_cast<long long>(Hkv) * __ldcg(rowstart + N);
+  const long long b0 = share_start(c, T, P), b1 = share_start(c + 1, T, P);
+  if (b0 >= b1) return;
   __syncthreads();
   const Guard guard{&ctl.abort, status, limit_ns};
 
@@ -668,8 +674,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
     ++issued;
   };
   if (tid == 0) {
-    tma_prefetch_desc(&mk);
-    tma_prefetch_desc(&mv);
     pk.begin(rowstart, N, Hkv, b0, b1, bits, H, g, W);
     for (int i = 0; i < kDecStages; ++i) issue_next();
   }
@@ -704,8 +708,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
     const uint32_t* hrow = bits + (static_cast<long long>(n) * H + kvh * g) * W;
     for (int w = cs.Ja >> 5; ok && w <= (cs.Jb - 1) >> 5; ++w) {
       // the lane's two heads' kept bits in this word, and the group's union
-      const uint32_t hb0 = 2 * tig < g ? __ldg(hrow + static_cast<long long>(2 * tig) * W + w) : 0u;
-      const uint32_t hb1 = 2 * tig + 1 < g ? __ldg(hrow + static_cast<long long>(2 * tig + 1) * W + w) : 0u;
+      const uint32_t hb0 = 2 * tig < g ? __ldcg(hrow + static_cast<long long>(2 * tig) * W + w) : 0u;
+      const uint32_t hb1 = 2 * tig + 1 < g ? __ldcg(hrow + static_cast<long long>(2 * tig + 1) * W + w) : 0u;
       uint32_t rem = group_word(bits, cs, H, g, W, w);
       while (rem) {
         const int jw = __ffs(static_cast<int>(rem)) - 1;
@@ -841,6 +845,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
     }
     more = cs.next();
   }
+  grid_dependents_launch();
   // copies still in flight land before the CTA exits (only after a wait ran out
   // can any be left)
   if (tid == 0) {
@@ -871,11 +876,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const float
   const int nthr = g * D / 4, groups = kDecThreads / nthr;
   const int grp = tid / nthr, e0 = 4 * (tid % nthr);
   const int hm = e0 / D, col = e0 % D;
-  const int nbl = __ldg(rowstart + n + 1) - __ldg(rowstart + n);
+  // the attention's partials (the grid ahead, launched so that this one may
+  // start early) are read only past this point, through L2
+  grid_dependency_wait();
+  const int nbl = __ldcg(rowstart + n + 1) - __ldcg(rowstart + n);
   float Mx = -INFINITY, L = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
   if (nbl > 0) {
-    const long long T = static_cast<long long>(Hkv) * __ldg(rowstart + N);
-    const long long s0 = static_cast<long long>(Hkv) * __ldg(rowstart + n) + static_cast<long long>(kvh) * nbl;
+    const long long T = static_cast<long long>(Hkv) * __ldcg(rowstart + N);
+    const long long s0 = static_cast<long long>(Hkv) * __ldcg(rowstart + n) + static_cast<long long>(kvh) * nbl;
     const int clo = share_owner(s0, T, P), chi = share_owner(s0 + nbl - 1, T, P);
     const int per = (chi - clo + 1 + groups - 1) / groups;
     const int g0 = clo + grp * per, g1 = min(g0 + per, chi + 1);
@@ -892,10 +900,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const float
         const int cc = base + u;
         const bool use = cc < g1 && (all_full || share_start(cc, T, P) != share_start(cc + 1, T, P));
         const float* pc = pr + static_cast<long long>(use ? cc : clo) * cs_stride;
-        mk[u] = __ldg(pc);
-        lk[u] = __ldg(pc + 1);
-        ok[u][0] = __ldg(reinterpret_cast<const float2*>(pc + 2 + col));
-        ok[u][1] = __ldg(reinterpret_cast<const float2*>(pc + 4 + col));
+        mk[u] = __ldcg(pc);
+        lk[u] = __ldcg(pc + 1);
+        ok[u][0] = __ldcg(reinterpret_cast<const float2*>(pc + 2 + col));
+        ok[u][1] = __ldcg(reinterpret_cast<const float2*>(pc + 4 + col));
         if (!use) mk[u] = -INFINITY;
       }
       float bm = Mx;
@@ -992,13 +1000,26 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
   static std::atomic<uint64_t> smem_set{0};
   if ((e = set_smem_limit_once(decode_attn_kernel<BN, D>, C::kSmem, smem_set)) != cudaSuccess) return e;
   const int P = std::max(1, std::min(sms, kDecAttnCTAs));
-  decode_attn_kernel<BN, D><<<P, kDecThreads, C::kSmem, stream>>>(
-      mk, mv, static_cast<const __nv_bfloat16*>(q), lens, w.rowstart, w.bits, N, Lmax, H, Hkv, W, sl2, w.part,
-      g.status, g.limit_ns);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  decode_combine_kernel<D><<<static_cast<unsigned>(N) * Hkv, kDecThreads, 0, stream>>>(
-      w.part, w.rowstart, N, H, Hkv, P, static_cast<__nv_bfloat16*>(o));
-  return cudaGetLastError();
+  // attention and combine may start while the grid ahead finishes (programmatic
+  // dependent launch); each waits for it before reading what it wrote
+  cudaLaunchAttribute early[1];
+  early[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  early[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(P);
+  lc.blockDim = dim3(kDecThreads);
+  lc.dynamicSmemBytes = C::kSmem;
+  lc.stream = stream;
+  lc.attrs = early;
+  lc.numAttrs = 1;
+  if ((e = cudaLaunchKernelEx(&lc, decode_attn_kernel<BN, D>, mk, mv, static_cast<const __nv_bfloat16*>(q), lens,
+                              static_cast<const int32_t*>(w.rowstart), static_cast<const uint32_t*>(w.bits), N, Lmax,
+                              H, Hkv, W, sl2, w.part, g.status, g.limit_ns)) != cudaSuccess)
+    return e;
+  lc.gridDim = dim3(static_cast<unsigned>(N) * Hkv);
+  lc.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&lc, decode_combine_kernel<D>, static_cast<const float*>(w.part),
+                            static_cast<const int32_t*>(w.rowstart), N, H, Hkv, P, static_cast<__nv_bfloat16*>(o));
 }
 
 }  // namespace

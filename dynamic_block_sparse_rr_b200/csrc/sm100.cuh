@@ -29,6 +29,15 @@ __device__ __forceinline__ uint64_t global_ns() {
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
+// Programmatic dependent launch.  A grid launched with programmatic stream
+// serialization may start while the grid ahead of it in the stream still runs;
+// grid_dependency_wait() returns once that grid has completed and its memory
+// operations are visible (at once for a grid launched without the attribute),
+// and grid_dependents_launch() lets the next such grid start once every CTA of
+// this grid has called it or exited.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
