@@ -40,6 +40,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <stdlib.h>
+
 #include <algorithm>
 #include <atomic>
 
@@ -491,6 +493,7 @@ struct DecAttnCfg {
 
 struct DecAttnCtrl {
   uint64_t full[kDecStages];
+  uint64_t never;                          // fault injection: a barrier nothing arrives on
   int abort;
   float2 ml[kDecWarps][8];                 // warp partials: (max, sum) per head
   __nv_bfloat16 p[kDecWarps][8][24];       // per warp: P of its 16 keys, [head][key] (rows padded)
@@ -625,7 +628,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
     const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lens, const int32_t* __restrict__ rowstart,
     const uint32_t* __restrict__ bits, int N, int Lmax, int H, int Hkv, int W, float sl2, float* __restrict__ part,
-    unsigned int* status, uint64_t limit_ns) {
+    unsigned int* status, uint64_t limit_ns, int inject_stall) {
   using C = DecAttnCfg<BN, D>;
   constexpr int kKeyWarps = BN / 16;  // warps that own keys (8 at B = 128, 4 at B = 64)
   constexpr int kDSteps = D / 16;     // k-steps of S (over d)
@@ -642,6 +645,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
   const int g = H / Hkv;
   if (tid == 0) {
     for (int st = 0; st < kDecStages; ++st) mbar_init(smem_u32(&ctl.full[st]), 1);
+    mbar_init(smem_u32(&ctl.never), 1);
     ctl.abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&mk);
@@ -680,6 +684,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(
 
   const int mi = lane >> 3, ri = lane & 7;   // ldmatrix: this lane's matrix and row
   bool ok = true;
+  // Injected fault (tests only): thread 0 waits on a barrier that nothing arrives
+  // on; the bounded wait gives up, and the CTA takes its abort path.
+  if (inject_stall && tid == 0) ok = wait_bar(smem_u32(&ctl.never), 0, guard, 9);
+  ok = __syncthreads_and(ok);
   int seq = 0;   // kept blocks consumed
   SegWalk cs;
   bool more = cs.begin(rowstart, N, Hkv, b0, b1);
@@ -1012,9 +1020,13 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const i
   lc.stream = stream;
   lc.attrs = early;
   lc.numAttrs = 1;
+  // RR_DEBUG_STALL_WAIT=1 injects a wait that never completes (tests of the
+  // bounded-wait path); unset in normal use.
+  const char* inj = getenv("RR_DEBUG_STALL_WAIT");
+  const int inject = (inj && inj[0] == '1') ? 1 : 0;
   if ((e = cudaLaunchKernelEx(&lc, decode_attn_kernel<BN, D>, mk, mv, static_cast<const __nv_bfloat16*>(q), lens,
                               static_cast<const int32_t*>(w.rowstart), static_cast<const uint32_t*>(w.bits), N, Lmax,
-                              H, Hkv, W, sl2, w.part, g.status, g.limit_ns)) != cudaSuccess)
+                              H, Hkv, W, sl2, w.part, g.status, g.limit_ns, inject)) != cudaSuccess)
     return e;
   lc.gridDim = dim3(static_cast<unsigned>(N) * Hkv);
   lc.dynamicSmemBytes = 0;

@@ -56,3 +56,38 @@ def test_wait_timeout_is_reported_and_context_survives(rr):
     O_ref = oracle.sparse_attention(Q, K, V, c, i, B, rows=[(0, 0), (3, 17), (H - 1, L // B - 1)])
     mx, mean = output_errors(o.float().cpu().numpy(), O_ref)
     assert mx <= 2e-2 and mean <= 2e-3
+
+
+def test_decode_wait_timeout_is_reported_and_context_survives(rr):
+    """The same injection in the decode step: every attention CTA's first wait
+    runs out, its rows get empty partials (zero outputs), the status reads
+    RR_ETIMEOUT, and the next call is correct again."""
+    N, Lmax, H, Hkv, d, B, S, tau = 2, 1024, 8, 2, 128, 128, 16, 0.9
+    lens = [1024, 700]
+    qs, ks, vs = [], [], []
+    for n in range(N):
+        q, k, v = gen.make_qkv(Lmax, H, Hkv, d, gen.PLANTED, 21 + n)
+        qs.append(gen.bf16_bits_to_f32(q)[lens[n] - 1])
+        ks.append(gen.bf16_bits_to_f32(k))
+        vs.append(gen.bf16_bits_to_f32(v))
+    Q, K, V = np.stack(qs), np.stack(ks), np.stack(vs)
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).cuda()
+    qd, kd, vd = to(Q), to(K), to(V)
+    ld = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ws = torch.empty(rr.decode_workspace_size(N, Lmax, H, Hkv, d, B, S), dtype=torch.uint8, device="cuda")
+    prev = rr.set_wait_limit_ns(20_000_000)
+    os.environ["RR_DEBUG_STALL_WAIT"] = "1"
+    try:
+        o, _, _ = rr.decode(qd, kd, vd, ld, B, S, tau, ws=ws)
+        status = rr.check_status(ws)
+    finally:
+        del os.environ["RR_DEBUG_STALL_WAIT"]
+        rr.set_wait_limit_ns(prev)
+    assert status == rr.RR_ETIMEOUT
+    assert not torch.any(o.float() != 0)
+    o, count, idx = rr.decode(qd, kd, vd, ld, B, S, tau, ws=ws)
+    assert rr.check_status(ws) == rr.RR_OK
+    og, c, i = o.float().cpu().numpy(), count.cpu().numpy(), idx.cpu().numpy()
+    for n in range(N):
+        ref = oracle.decode_attention(Q[n], K[n], V[n], lens[n] - 1, [i[n, h, :c[n, h]] for h in range(H)], B)
+        assert np.abs(og[n] - ref).max() <= 2e-2
