@@ -104,8 +104,10 @@ def test_decode_llama_shaped(rr, tau):
     run_case(rr, len(lens), 4096, 8, 2, 128, 128, 16, tau, lens)
 
 
-@pytest.mark.parametrize("B,d,S", [(64, 64, 4), (64, 128, 8), (128, 64, 32)])
+@pytest.mark.parametrize("B,d,S", [(64, 64, 4), (64, 128, 8), (128, 64, 32), (128, 128, 1), (64, 64, 64)])
 def test_decode_block_and_head_sizes(rr, B, d, S):
+    """B, d in {64, 128} and strides per block r = B/S from 1 (one sampled key
+    per block) to 128 (every key sampled)."""
     lens = [2048, 1000, 65]
     run_case(rr, len(lens), 2048, 4, 1, d, B, S, 0.9, lens, structure=gen.PLANTED_BAND, seed=3)
 
