@@ -550,11 +550,55 @@ def measure_decode(args, rr, cfg, tau, qd, kd, vd, dev, stream):
                 "hbm": {"bytes": byts["total"], "gbs": gbs, "frac_of_hbm": gbs / peak, "peak_gbs": peak,
                         "parts": byts}}
 
+    # the step captured once in a CUDA graph and replayed, as a serving loop would;
+    # and the latency of one step with the host waiting for it, eager and replayed
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(2):
+            rr.decode(qq, kc, vc, ld, B, S, tau, out=out, count=cnt, idx=idx, ws=ws)
+    stream.wait_stream(side)
+    with torch.cuda.graph(graph):
+        rr.decode(qq, kc, vc, ld, B, S, tau, out=out, count=cnt, idx=idx, ws=ws)
+
+    def timed_graph(reps=10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    def latency(fn, n=30):
+        ts = []
+        for _ in range(n):
+            torch.cuda.synchronize(dev)
+            t0 = time.perf_counter()
+            fn()
+            torch.cuda.synchronize(dev)
+            ts.append(time.perf_counter() - t0)
+        return statistics.median(ts) * 1e3
+
+    timed_graph(3)
+    graph_ms = statistics.median([timed_graph() for _ in range(3)])
+    lat_eager = latency(lambda: rr.decode(qq, kc, vc, ld, B, S, tau, out=out, count=cnt, idx=idx, ws=ws,
+                                          stream=stream))
+    lat_graph = latency(graph.replay)
+    if rr.check_status(ws) != rr.RR_OK:
+        raise RuntimeError("device-side status of the replayed decode step")
+    del graph
+
     res = {"what": "rr_decode: one new token per sequence over its KV cache (search, block-sparse attention "
                    "with the partials merged); caches are copies of this layer, sequence n holds L - 1000 n keys",
            "batch": Nd, "dense_us_per_step": dense_ms * 1e3}
     res.update(summary(cnt, idx, ms))
     res["gqa_mask"] = summary(cnt_g, idx_g, g_ms)
+    res["cuda_graph"] = {"us_per_step": graph_ms * 1e3,
+                         "latency_us": {"eager": lat_eager * 1e3, "graph": lat_graph * 1e3},
+                         "note": "one step captured in a CUDA graph and replayed back to back; latency is the "
+                                 "host-clock median of one step with a synchronize on each side"}
     del kc, vc, ws
     torch.cuda.empty_cache()
     return res

@@ -252,3 +252,36 @@ def test_decode_llama128k_last_token(rr):
     print({"visited": float(count.sum()) / (H * (t // B + 1)), "max_err": float(err.max()),
            "mean_err": float(err.mean())})
     assert err.max() <= MAX_ERR and err.mean() <= MEAN_ERR
+
+
+def test_decode_replays_from_a_cuda_graph(rr):
+    """A decode step captured in a CUDA graph (memset, search, attention and
+    combine with their programmatic launch edges) and replayed gives the
+    eager call's lists and outputs bit for bit."""
+    N, Lmax, H, Hkv, d, B, S, tau = 3, 2048, 8, 2, 128, 128, 16, 0.9
+    Qs, K, V = _make(N, Lmax, H, Hkv, d, gen.PLANTED, 43)
+    lens = [2048, 1500, 130]
+    q = _bf16(np.stack([Qs[n][lens[n] - 1] for n in range(N)])).cuda()
+    kd, vd = _bf16(K).cuda(), _bf16(V).cuda()
+    ld = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ws = torch.empty(rr.decode_workspace_size(N, Lmax, H, Hkv, d, B, S), dtype=torch.uint8, device="cuda")
+    o_e, c_e, i_e = rr.decode(q, kd, vd, ld, B, S, tau, ws=ws)
+    o, c, i = torch.empty_like(o_e), torch.empty_like(c_e), torch.empty_like(i_e)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        rr.decode(q, kd, vd, ld, B, S, tau, out=o, count=c, idx=i, ws=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    o.zero_()
+    c.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        rr.decode(q, kd, vd, ld, B, S, tau, out=o, count=c, idx=i, ws=ws)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert rr.check_status(ws) == rr.RR_OK
+    assert torch.equal(o, o_e) and torch.equal(c, c_e)
+    for n in range(N):
+        for h in range(H):
+            assert torch.equal(i[n, h, :c[n, h]], i_e[n, h, :c_e[n, h]])
