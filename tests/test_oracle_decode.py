@@ -180,8 +180,33 @@ def test_group_mask_shares_lists_and_reaches_tau():
     assert all(np.array_equal(a, b) for a, b in zip(s1, s2)) and np.allclose(o1, o2)
 
 
+def test_group_mask_groups_the_heads_of_each_kv_head():
+    """Planted keys: each head's mass sits on a block of its own (one key per
+    head at that head's own offset, on its own kv head, logit 30).  With one
+    list per GQA group and tau = 0.9, a group's list must hold exactly the
+    planted blocks of the heads that share its kv head (each carries 1/g of the
+    group mass) and the current block; grouping other heads together, or
+    selecting on one head's mass, gives other sets."""
+    L, H, Hkv, d, B, S = 1024, 6, 3, 16, 32, 8
+    t = L - 1
+    g, r = H // Hkv, B // S
+    q = np.zeros((H, d))
+    q[:, 0] = 1.0
+    K = np.zeros((L, Hkv, d))
+    j_of = {h: 3 + 11 * h for h in range(H)}
+    for h in range(H):
+        K[j_of[h] * S + h % S, h // g, 0] = 30.0 * math.sqrt(d)
+    V = np.zeros((L, Hkv, d))
+    _, sel, _, _ = oracle.rr_decode(q, K, V, t, B, S, 0.9, gqa_mask=True)
+    for h in range(H):
+        c = h // g
+        want = {j_of[u] // r for u in range(c * g, (c + 1) * g)} | {t // B}
+        assert set(sel[h].tolist()) == want, (h, sel[h], want)
+
+
 # ------------------------------------------------------------ planted mistakes
-_orig = {n: getattr(oracle, n) for n in ("decode_positions", "decode_select", "decode_attention")}
+_orig = {n: getattr(oracle, n) for n in ("decode_positions", "decode_select", "decode_attention",
+                                         "decode_group_mass")}
 
 
 def _positions_past_t(t, h, S):
@@ -216,6 +241,21 @@ def _attention_whole_block(q, K, V, t, blocks, B):
     return out
 
 
+def _group_mass_by_modulo(M, Hkv):
+    H, n = M.shape
+    g = H // Hkv
+    out = np.zeros_like(M)
+    for h in range(H):
+        out[h] = M[[u for u in range(H) if u % Hkv == h % Hkv]].sum(axis=0)
+    return out
+
+
+def _group_mass_first_head(M, Hkv):
+    H, n = M.shape
+    g = H // Hkv
+    return np.repeat(M[::g], g, axis=0)
+
+
 DECODE_PINS = [
     lambda: test_tau_one_equals_dense_decode_attention(37),
     lambda: test_stride_one_mass_equals_exact_attention_mass(100),
@@ -223,6 +263,7 @@ DECODE_PINS = [
     test_keys_sampled_past_the_query_do_not_count,
     test_query_before_its_heads_first_sample,
     lambda: test_selection_brute_force_and_current_block(0.7),
+    test_group_mask_groups_the_heads_of_each_kv_head,
 ]
 
 DECODE_MUTANTS = {
@@ -232,6 +273,8 @@ DECODE_MUTANTS = {
                                     if t >= h else np.zeros(0, np.int64)),
     "current block not protected": ("decode_select", _select_unprotected),
     "attention reads keys past the query": ("decode_attention", _attention_whole_block),
+    "group mask groups heads by h mod Hkv": ("decode_group_mass", _group_mass_by_modulo),
+    "group mask selects on the group's first head only": ("decode_group_mass", _group_mass_first_head),
 }
 
 
