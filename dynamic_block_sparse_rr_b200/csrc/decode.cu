@@ -18,11 +18,14 @@
 //                          scores to the workspace, the run's max and block
 //                          masses on that max.  The CTA that finishes a row
 //                          last puts the row's masses on one scale and runs
-//                          Top-tau by bisection over the mass bits with
-//                          block-wide sums of fixed-point units (the prefill
-//                          rule); list and a bitmap of the kept blocks out.
-//                          One CTA also writes the prefix of the sequences'
-//                          block counts;
+//                          Top-tau on fixed-point units of the row total (the
+//                          prefill rule), its threshold found by four passes
+//                          over 8-bit digits of the mass bits; list and a
+//                          bitmap of the kept blocks out.  One CTA also writes
+//                          the prefix of the sequences' block counts;
+//   decode_group_select_kernel  (one list per GQA group only) one CTA per
+//                          (sequence, kv head): Top-tau on the group's summed
+//                          masses, the list written to every head of the group;
 //   decode_attn_kernel     one persistent CTA per SM over an equal share of the
 //                          flattened (sequence, kv head, causal key block)
 //                          space: a kept block's K and V tiles come in once by
@@ -39,7 +42,6 @@
 //                          CTAs that shared the row merged into the output.
 #include <cuda_bf16.h>
 #include <math.h>
-
 #include <stdlib.h>
 
 #include <algorithm>
@@ -148,9 +150,9 @@ struct DecSearchShared {
 };
 
 // Top-tau over the nb = Jt + 1 block masses in mass[] (shared memory), as in
-// prefill (fixed-point units of the row total, the threshold by bisection over
-// the mass bits with block-wide sums, equal masses to the lower J), plus the
-// current block Jt.  wbits (shared memory, ceil(nb/32) words) collects the
+// prefill (fixed-point units of the row total; the threshold, the largest mass
+// whose masses at or above it reach the target, found digit by digit of the
+// mass bits; equal masses to the lower J), plus the current block Jt.  wbits (shared memory, ceil(nb/32) words) collects the
 // bitmap.  The ascending list goes to rep consecutive rows of out (row stride
 // out_stride), the bitmap to rep consecutive rows of obits (W words each), the
 // count to count[0 .. rep).  Called by every thread of the CTA.
